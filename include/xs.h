@@ -1,0 +1,147 @@
+/*
+ * xs.h -- C ABI of libxs.so: non-causal DiT self-attention fused, tile by tile, with the
+ * Ulysses post-attention All-to-All, for NVIDIA B200 (sm_100a).
+ *
+ * The operation (page "X-Stage: An Overlooked Pipeline Stage for Communication-Computation
+ * Overlap in DiT Inference": abstract, and the explainer's "Technisches Resuemee" ->
+ * "Zentrale Beitraege" -> "FlashAttention-A2A (Piggybacking)"):
+ *   O[b,h,i,:] = softmax_j(scale * q[b,h,i,:] . k[b,h,j,:]) v[b,h,j,:]   (non-causal)
+ * followed by the post-attention All-to-All that moves every output row into the sequence
+ * shard of its destination rank,
+ *   dest[r][b, s_local, h, :] = O[b, h, r*S/P + s_local, :].
+ * In the fused call the owner of a finished output tile stores it straight into the
+ * destination slabs and goes on with its next tile; no warp or SM is set aside for the
+ * exchange.  On one GPU the P ranks are P slabs in local memory.
+ *
+ * Conventions shared by every call:
+ *  - Tensors are bf16 stored as 16-bit words, row-major and contiguous.  q, k, v and the
+ *    head-major output use [B, H, S, D]; each destination slab uses [B, S/P, H, D].
+ *  - Every pointer named "device" points to memory the caller allocated on the current
+ *    CUDA device, 16-byte aligned.  The caller owns all buffers; the library never
+ *    allocates, frees or keeps device memory and never synchronises.
+ *  - All work is enqueued on `stream` (NULL = legacy default stream) and runs
+ *    asynchronously.  Host-detectable errors return before anything is enqueued.
+ *  - `dev_status` (nullable) is a device int the kernels set to a non-zero xs_status when a
+ *    bounded on-device wait gives up (XS_ERR_TIMEOUT).  The caller zeroes it before the
+ *    call and reads it after its own synchronisation.
+ *  - Supported shapes: B, H, S, D, P >= 1; H % P == 0 and S % P == 0 (Ulysses sharding);
+ *    D % 8 == 0 and 8 <= D <= 128; P <= XS_MAX_RANKS.  S need not be a multiple of the
+ *    128-row tile: ragged tails are masked.
+ */
+#ifndef XS_H_
+#define XS_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define XS_API __attribute__((visibility("default")))
+#else
+#define XS_API
+#endif
+
+#define XS_VERSION 100   /* 1.0.0 */
+#define XS_MAX_RANKS 16
+
+typedef enum {
+  XS_OK = 0,
+  XS_ERR_INVALID_ARG = 1, /* null/misaligned/overlapping pointers, non-positive sizes   */
+  XS_ERR_UNSUPPORTED = 2, /* shape outside the supported set (see conventions)          */
+  XS_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (launch, tensor map, ...) */
+  XS_ERR_TIMEOUT = 4      /* written to *dev_status by a bounded on-device wait          */
+} xs_status;
+
+/* Problem shape.  B batch, H heads, S sequence length, D head dim, P Ulysses ranks. */
+typedef struct {
+  int B, H, S, D, P;
+} xs_shape;
+
+struct CUstream_st;
+typedef struct CUstream_st *xs_stream_t; /* the same handle as cudaStream_t */
+
+/*
+ * Fused attention + post-attention All-to-All (the hot path).
+ *   q, k, v   : device, [B, H, S, D] bf16.
+ *   dest      : HOST array of P device pointers; dest[r] is rank r's slab [B, S/P, H, D].
+ *               Slabs must not overlap one another or q, k, v.
+ *   scale     : softmax scale; <= 0 selects 1/sqrt(D) with the true D.
+ * Numerics: bf16 operands, fp32 accumulation of Q K^T and P V, probabilities rounded to
+ * bf16 before P V, fp32 row sums of those rounded probabilities, output rounded to bf16
+ * (nearest even).
+ * Returns XS_OK once the work is enqueued; errors as listed in xs_status.
+ */
+XS_API xs_status xs_attn_a2a_fused(const void *q, const void *k, const void *v, void *const *dest,
+                            xs_shape shape, float scale, xs_stream_t stream, int *dev_status);
+
+/*
+ * Attention only, head-major output: out[b,h,s,:] (device, [B, H, S, D] bf16).  The same
+ * kernel and arithmetic as xs_attn_a2a_fused, so out re-laid by xs_a2a_relayout equals the
+ * fused result bit for bit.  First half of the serial baseline the pages compare against
+ * ("over serial execution", same item of the explainer).  P is only range-checked here.
+ */
+XS_API xs_status xs_attn(const void *q, const void *k, const void *v, void *out, xs_shape shape,
+                  float scale, xs_stream_t stream, int *dev_status);
+
+/*
+ * The post-attention All-to-All as a separate pass (second half of the serial baseline):
+ *   dest[r][b, s_local, h, :] = src[b, h, r*S/P + s_local, :]
+ * src: device [B, H, S, D] 16-bit words; dest: host array of P device slab pointers.  A pure
+ * copy: every destination word equals its source word.
+ */
+XS_API xs_status xs_a2a_relayout(const void *src, void *const *dest, xs_shape shape,
+                          xs_stream_t stream);
+
+/*
+ * Burst-Gap store microbenchmark (explainer, "Methodik: Die X-Stage-Abstraktion und das
+ * Burst-Gap-Modell": sender-visible issue time T_iss(G; K, V) of a burst of volume V from K
+ * producers separated by a compute gap G).  Each of `producers` CTAs repeats n_bursts times:
+ * issue its share (burst_bytes / producers) of 16-byte stores into `scratch`, record when
+ * the last of its threads has issued, then run a dependent FMA chain of about gap_cycles
+ * cycles.  Nothing waits for the stores to complete: the measured time is what the issuer
+ * sees.
+ *   scratch       : device buffer of scratch_bytes bytes (stored to, never read).
+ *                   Bursts walk through it cyclically, so a buffer larger than L2 makes the
+ *                   stores drain to HBM.
+ *   stamps        : device, [producers, n_bursts, 4] uint64 per burst: SM clock at burst
+ *                   start, SM clock when the CTA finished issuing, SM clock at gap end,
+ *                   global timer (ns) at burst start.
+ * Limits: burst_bytes % (16 * producers) == 0; each producer's share >= 16 bytes and
+ * <= scratch_bytes / producers; 1 <= producers <= 4096; 1 <= n_bursts <= 1 << 20;
+ * 0 <= gap_cycles <= 1 << 30; threads_per_producer in {32, 64, ..., 1024}.
+ */
+typedef struct {
+  long long burst_bytes;    /* V: aggregate bytes per burst over all producers */
+  int producers;            /* K: number of producer CTAs                        */
+  long long gap_cycles;     /* G: compute gap after each burst, in SM cycles     */
+  int n_bursts;             /* bursts per producer                               */
+  int threads_per_producer; /* CTA size                                          */
+} xs_burst_cfg;
+
+XS_API xs_status xs_burst_probe(void *scratch, long long scratch_bytes, xs_burst_cfg cfg,
+                         unsigned long long *stamps, xs_stream_t stream);
+
+/*
+ * Self-test of the bounded on-device wait used by every kernel in this library: launches
+ * one thread that waits on a shared-memory barrier nothing ever arrives at, gives up after
+ * limit_ns nanoseconds of global time (1e3 <= limit_ns <= 1e10) and writes XS_ERR_TIMEOUT
+ * to *dev_status (device, required).  The context stays usable afterwards.
+ */
+XS_API xs_status xs_selftest_bounded_wait(int *dev_status, long long limit_ns, xs_stream_t stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+XS_API const char *xs_get_error_string(xs_status status);
+
+/* Library version, XS_VERSION of the build. */
+XS_API int xs_version(void);
+
+/* Text of the last error the calling thread got from this library (static per thread). */
+XS_API const char *xs_last_error_detail(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* XS_H_ */

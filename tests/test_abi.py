@@ -1,0 +1,118 @@
+"""The C-ABI library on the host (CPU only): it builds, loads, exports every symbol that
+``include/xs.h`` declares, and rejects bad arguments with the documented codes before any
+CUDA call.  No kernel is launched here.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import ulysses_attention_output_b200 as xs
+from ulysses_attention_output_b200 import build as xs_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    xs_build.build()
+    return xs.load()
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"XS_API\s+[\w\s\*]+?\b(xs_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert {"xs_attn_a2a_fused", "xs_attn", "xs_a2a_relayout", "xs_burst_probe"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported by libxs.so"
+
+
+def test_version_and_strings(lib):
+    assert xs.version() == 100
+    for code, name in [(0, b"XS_OK"), (1, b"XS_ERR_INVALID_ARG"), (2, b"XS_ERR_UNSUPPORTED"),
+                       (3, b"XS_ERR_CUDA"), (4, b"XS_ERR_TIMEOUT")]:
+        assert lib.xs_get_error_string(code) == name
+
+
+FAKE = 0x7f0000000000  # never dereferenced: every call below fails validation first
+MB = 1 << 20
+
+
+def fused(lib, q, k, v, dests, shape, scale=0.0):
+    arr = (ctypes.c_void_p * max(1, len(dests)))(*dests) if dests is not None else None
+    return lib.xs_attn_a2a_fused(q, k, v, arr, xs.Shape(*shape), scale, None, None)
+
+
+@pytest.mark.parametrize("shape,code", [
+    ((1, 4, 256, 100, 2), xs.XS_ERR_UNSUPPORTED),   # D not a multiple of 8
+    ((1, 4, 256, 136, 2), xs.XS_ERR_UNSUPPORTED),   # D > 128
+    ((1, 3, 256, 64, 2), xs.XS_ERR_UNSUPPORTED),    # H % P != 0
+    ((1, 4, 255, 64, 2), xs.XS_ERR_UNSUPPORTED),    # S % P != 0
+    ((1, 32, 256, 64, 32), xs.XS_ERR_UNSUPPORTED),  # P > 16
+    ((0, 4, 256, 64, 2), xs.XS_ERR_INVALID_ARG),    # empty batch
+    ((1, 4, 256, 64, 0), xs.XS_ERR_INVALID_ARG),    # no ranks
+])
+def test_fused_rejects_shapes(lib, shape, code):
+    dests = [FAKE + 100 * MB * (r + 1) for r in range(max(shape[4], 1))]
+    assert fused(lib, FAKE, FAKE + 30 * MB, FAKE + 60 * MB, dests, shape) == code
+
+
+def test_fused_rejects_pointers(lib):
+    shape = (1, 4, 256, 64, 2)
+    good = [FAKE + 100 * MB, FAKE + 200 * MB]
+    assert fused(lib, 0, FAKE + 30 * MB, FAKE + 60 * MB, good, shape) == xs.XS_ERR_INVALID_ARG
+    assert fused(lib, FAKE + 8, FAKE + 30 * MB, FAKE + 60 * MB, good, shape) == xs.XS_ERR_INVALID_ARG
+    assert fused(lib, FAKE, FAKE + 30 * MB, FAKE + 60 * MB, None, shape) == xs.XS_ERR_INVALID_ARG
+    assert fused(lib, FAKE, FAKE + 30 * MB, FAKE + 60 * MB, [good[0], 0], shape) == xs.XS_ERR_INVALID_ARG
+    # overlapping slabs, slab overlapping an input
+    assert fused(lib, FAKE, FAKE + 30 * MB, FAKE + 60 * MB, [good[0], good[0] + 1024], shape) == xs.XS_ERR_INVALID_ARG
+    assert fused(lib, FAKE, FAKE + 30 * MB, FAKE + 60 * MB, [good[0], FAKE + 1024], shape) == xs.XS_ERR_INVALID_ARG
+    detail = lib.xs_last_error_detail().decode()
+    assert "overlaps" in detail
+
+
+def test_attn_and_relayout_reject(lib):
+    sh = xs.Shape(1, 4, 256, 64, 2)
+    assert lib.xs_attn(FAKE, FAKE + MB, FAKE + 2 * MB, 0, sh, 0.0, None, None) == xs.XS_ERR_INVALID_ARG
+    assert lib.xs_attn(FAKE, FAKE + MB, FAKE + 2 * MB, FAKE, sh, 0.0, None, None) == xs.XS_ERR_INVALID_ARG
+    arr = (ctypes.c_void_p * 2)(FAKE + 100 * MB, FAKE + 200 * MB)
+    assert lib.xs_a2a_relayout(0, arr, sh, None) == xs.XS_ERR_INVALID_ARG
+    assert lib.xs_a2a_relayout(FAKE, arr, xs.Shape(1, 4, 256, 60, 2), None) == xs.XS_ERR_UNSUPPORTED
+
+
+def test_probe_and_selftest_reject(lib):
+    cfg = xs.BurstCfg(4096, 4, 0, 8, 256)
+    assert lib.xs_burst_probe(0, 1 << 20, cfg, FAKE, None) == xs.XS_ERR_INVALID_ARG
+    assert lib.xs_burst_probe(FAKE, 1 << 20, xs.BurstCfg(4100, 4, 0, 8, 256), FAKE + 8 * MB, None) == xs.XS_ERR_INVALID_ARG
+    assert lib.xs_burst_probe(FAKE, 1024, cfg, FAKE + 8 * MB, None) == xs.XS_ERR_INVALID_ARG
+    assert lib.xs_burst_probe(FAKE, 1 << 20, xs.BurstCfg(4096, 4, 0, 8, 100), FAKE + 8 * MB, None) == xs.XS_ERR_INVALID_ARG
+    assert lib.xs_selftest_bounded_wait(0, 10 ** 6, None) == xs.XS_ERR_INVALID_ARG
+    assert lib.xs_selftest_bounded_wait(FAKE, 10, None) == xs.XS_ERR_INVALID_ARG
+
+
+def test_binding_has_no_fallback(monkeypatch, tmp_path):
+    """With the library missing, the binding raises instead of computing anything else."""
+    monkeypatch.setattr(xs, "_lib", None)
+    monkeypatch.setenv("XS_LIBRARY", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        xs.load()
+    monkeypatch.setattr(xs, "_lib", None)
+
+
+def test_product_never_imports_oracle():
+    pkg = os.path.join(ROOT, "ulysses_attention_output_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, fn)).read()
+                assert "import oracle" not in text and "from oracle" not in text, fn
+                assert "xs_oracle" not in text, fn

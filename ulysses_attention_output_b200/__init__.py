@@ -1,0 +1,250 @@
+"""Python binding of libxs.so: fused DiT attention + Ulysses post-attention All-to-All (B200).
+
+Argument marshalling only.  Every step of the computation runs in the CUDA kernels of
+``libxs.so`` (declared in ``include/xs.h``); PyTorch only supplies device memory and streams.
+There is no fallback: if the library is missing or a call fails, these functions raise.
+
+Calls (same names as the C ABI, without the ``xs_`` prefix):
+
+* :func:`attn_a2a_fused` -- attention fused with the post-attention exchange into P slabs.
+* :func:`attn`           -- attention with a head-major output.
+* :func:`a2a_relayout`   -- the exchange as a separate pass (serial baseline).
+* :func:`burst_probe`    -- Burst-Gap store microbenchmark.
+* :func:`selftest_bounded_wait` -- exercises the bounded on-device wait.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+__all__ = [
+    "XsError", "XS_OK", "XS_ERR_INVALID_ARG", "XS_ERR_UNSUPPORTED", "XS_ERR_CUDA", "XS_ERR_TIMEOUT",
+    "library_path", "load", "version", "attn_a2a_fused", "attn", "a2a_relayout", "burst_probe",
+    "selftest_bounded_wait", "alloc_dest", "HostPipeline", "attention_flops",
+]
+
+XS_OK, XS_ERR_INVALID_ARG, XS_ERR_UNSUPPORTED, XS_ERR_CUDA, XS_ERR_TIMEOUT = 0, 1, 2, 3, 4
+XS_MAX_RANKS = 16
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_lock = threading.Lock()
+_lib = None
+
+
+class XsError(RuntimeError):
+    """A libxs call returned a non-zero status."""
+
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{_STATUS_NAMES.get(status, status)}: {detail}")
+        self.status = status
+
+
+_STATUS_NAMES = {0: "XS_OK", 1: "XS_ERR_INVALID_ARG", 2: "XS_ERR_UNSUPPORTED", 3: "XS_ERR_CUDA",
+                 4: "XS_ERR_TIMEOUT"}
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("S", ctypes.c_int), ("D", ctypes.c_int),
+                ("P", ctypes.c_int)]
+
+
+class BurstCfg(ctypes.Structure):
+    _fields_ = [("burst_bytes", ctypes.c_longlong), ("producers", ctypes.c_int),
+                ("gap_cycles", ctypes.c_longlong), ("n_bursts", ctypes.c_int),
+                ("threads_per_producer", ctypes.c_int)]
+
+
+def library_path() -> str:
+    return os.environ.get("XS_LIBRARY", os.path.join(_HERE, "libxs.so"))
+
+
+def load():
+    """Load libxs.so (once).  Raises if it has not been built: there is no other path."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with "
+                               "`python -m ulysses_attention_output_b200.build`")
+        lib = ctypes.CDLL(path)
+        vp, c_int, c_float = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        vpp = ctypes.POINTER(ctypes.c_void_p)
+        ip = ctypes.c_void_p  # device int*
+        lib.xs_attn_a2a_fused.argtypes = [vp, vp, vp, vpp, Shape, c_float, vp, ip]
+        lib.xs_attn.argtypes = [vp, vp, vp, vp, Shape, c_float, vp, ip]
+        lib.xs_a2a_relayout.argtypes = [vp, vpp, Shape, vp]
+        lib.xs_burst_probe.argtypes = [vp, ctypes.c_longlong, BurstCfg, vp, vp]
+        lib.xs_selftest_bounded_wait.argtypes = [ip, ctypes.c_longlong, vp]
+        for fn in (lib.xs_attn_a2a_fused, lib.xs_attn, lib.xs_a2a_relayout, lib.xs_burst_probe,
+                   lib.xs_selftest_bounded_wait):
+            fn.restype = c_int
+        lib.xs_get_error_string.argtypes = [c_int]
+        lib.xs_get_error_string.restype = ctypes.c_char_p
+        lib.xs_last_error_detail.restype = ctypes.c_char_p
+        lib.xs_version.restype = c_int
+        _lib = lib
+        return lib
+
+
+def version() -> int:
+    return int(load().xs_version())
+
+
+def _check(rc: int):
+    if rc != XS_OK:
+        detail = load().xs_last_error_detail().decode(errors="replace")
+        raise XsError(rc, detail)
+
+
+# ------------------------------------------------------------------ marshalling helpers
+def _stream_handle(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream or None
+    if isinstance(stream, int):
+        return stream or None
+    return stream.cuda_stream or None
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _bf16_cuda(name: str, t, shape=None):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
+        raise TypeError(f"{name} must hold 16-bit words (bf16), got {t.dtype}")
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _shape_of(q, P: int) -> Shape:
+    if q.dim() != 4:
+        raise ValueError("q must be [B, H, S, D]")
+    B, H, S, D = (int(x) for x in q.shape)
+    return Shape(B, H, S, D, int(P))
+
+
+def _dest_array(dest, shp: Shape):
+    if len(dest) != shp.P:
+        raise ValueError(f"need {shp.P} destination slabs, got {len(dest)}")
+    for r, d in enumerate(dest):
+        _bf16_cuda(f"dest[{r}]", d, (shp.B, shp.S // max(shp.P, 1), shp.H, shp.D))
+    arr = (ctypes.c_void_p * shp.P)(*[d.data_ptr() for d in dest])
+    return arr
+
+
+def attention_flops(B: int, H: int, S: int, D: int) -> int:
+    """Algorithmic FLOPs of one attention pass, 4*B*H*S^2*D (two S x S x D contractions)."""
+    return 4 * B * H * S * S * D
+
+
+# ------------------------------------------------------------------ calls
+def attn_a2a_fused(q, k, v, dest, scale: float | None = None, stream=None, status=None):
+    """Attention + post-attention All-to-All: fills ``dest[r]`` ([B, S/P, H, D]) for r < P."""
+    P = len(dest)
+    shp = _shape_of(q, P)
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _bf16_cuda(n, t, tuple(q.shape))
+    arr = _dest_array(dest, shp)
+    _check(load().xs_attn_a2a_fused(q.data_ptr(), k.data_ptr(), v.data_ptr(), arr, shp,
+                                    float(scale or 0.0), _stream_handle(stream), _ptr(status)))
+
+
+def attn(q, k, v, out, scale: float | None = None, stream=None, status=None, P: int = 1):
+    """Attention with head-major output ``out`` [B, H, S, D]."""
+    shp = _shape_of(q, P)
+    for n, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+        _bf16_cuda(n, t, tuple(q.shape))
+    _check(load().xs_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), shp,
+                          float(scale or 0.0), _stream_handle(stream), _ptr(status)))
+
+
+def a2a_relayout(src, dest, stream=None):
+    """Post-attention All-to-All as its own pass: head-major ``src`` -> P slabs ``dest``."""
+    P = len(dest)
+    shp = _shape_of(src, P)
+    _bf16_cuda("src", src)
+    arr = _dest_array(dest, shp)
+    _check(load().xs_a2a_relayout(src.data_ptr(), arr, shp, _stream_handle(stream)))
+
+
+def burst_probe(scratch, stamps, burst_bytes: int, producers: int, gap_cycles: int,
+                n_bursts: int, threads_per_producer: int = 256, stream=None):
+    """Burst-Gap microbenchmark; ``stamps`` is a uint64/int64 CUDA tensor [producers, n_bursts, 4]."""
+    import torch
+    if not scratch.is_cuda or not stamps.is_cuda:
+        raise ValueError("scratch and stamps must be CUDA tensors")
+    if stamps.dtype not in (torch.int64, torch.uint64) or stamps.numel() < producers * n_bursts * 4:
+        raise ValueError("stamps must be int64/uint64 with producers * n_bursts * 4 elements")
+    cfg = BurstCfg(int(burst_bytes), int(producers), int(gap_cycles), int(n_bursts),
+                   int(threads_per_producer))
+    nbytes = scratch.numel() * scratch.element_size()
+    _check(load().xs_burst_probe(scratch.data_ptr(), nbytes, cfg, stamps.data_ptr(),
+                                 _stream_handle(stream)))
+
+
+def selftest_bounded_wait(status, limit_ns: int, stream=None):
+    """Launch the bounded-wait self-test; ``status`` (int32 CUDA tensor) receives XS_ERR_TIMEOUT."""
+    _check(load().xs_selftest_bounded_wait(status.data_ptr(), int(limit_ns), _stream_handle(stream)))
+
+
+def alloc_dest(B: int, H: int, S: int, D: int, P: int, device=None, fill: float | None = None):
+    """P separately allocated destination slabs [B, S/P, H, D] bf16 (caller-owned memory)."""
+    import torch
+    if S % P:
+        raise ValueError("S must be divisible by P")
+    out = []
+    for _ in range(P):
+        t = torch.empty((B, S // P, H, D), dtype=torch.bfloat16, device=device)
+        if fill is not None:
+            t.fill_(fill)
+        out.append(t)
+    return out
+
+
+class HostPipeline:
+    """End-to-end call with host buffers: pinned host q/k/v in, pinned host slabs out.
+
+    ``run`` enqueues on one stream: three host-to-device copies, the fused kernel, and one
+    device-to-host copy per slab.  Device buffers are allocated once, here, by PyTorch.
+    """
+
+    def __init__(self, B: int, H: int, S: int, D: int, P: int, device=None, scale=None):
+        import torch
+        self.shape = (B, H, S, D)
+        self.P = P
+        self.scale = scale
+        dev = device or torch.device("cuda")
+        self.q = torch.empty(self.shape, dtype=torch.bfloat16, device=dev)
+        self.k = torch.empty_like(self.q)
+        self.v = torch.empty_like(self.q)
+        self.dest = alloc_dest(B, H, S, D, P, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    @property
+    def h2d_bytes(self) -> int:
+        return 3 * self.q.numel() * 2
+
+    @property
+    def d2h_bytes(self) -> int:
+        return sum(d.numel() * 2 for d in self.dest)
+
+    def run(self, q_host, k_host, v_host, dest_host, stream=None):
+        import torch
+        s = stream or torch.cuda.current_stream()
+        with torch.cuda.stream(s):
+            self.q.copy_(q_host, non_blocking=True)
+            self.k.copy_(k_host, non_blocking=True)
+            self.v.copy_(v_host, non_blocking=True)
+            attn_a2a_fused(self.q, self.k, self.v, self.dest, scale=self.scale, stream=s,
+                           status=self.status)
+            for dh, dd in zip(dest_host, self.dest):
+                dh.copy_(dd, non_blocking=True)

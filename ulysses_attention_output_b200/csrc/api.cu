@@ -1,0 +1,270 @@
+// api.cu -- the C ABI of libxs.so (declared in include/xs.h): argument checks, TMA tensor
+// maps and kernel launches.  No device memory is allocated, freed or kept here, and nothing
+// synchronises: every call only enqueues work on the caller's stream.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/xs.h"
+#include "xs_internal.cuh"
+
+namespace {
+
+thread_local char g_detail[512] = "";
+
+xs_status fail(xs_status code, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+xs_status ok() {
+  g_detail[0] = '\0';
+  return XS_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Range {
+  uintptr_t lo, hi;  // [lo, hi)
+};
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+
+// ------------------------------------------------------------------ driver entry point
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  std::call_once(g_encode_once, [] {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+// 3-D view {D, S, B*H} of a [B, H, S, D] bf16 tensor; box {64, 128, 1}; 128-byte swizzle;
+// out-of-range elements (D padding, rows past S) read as zero.
+bool make_qkv_map(CUtensorMap *m, const void *ptr, const xs_shape &s) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(s.D), static_cast<cuuint64_t>(s.S),
+                        static_cast<cuuint64_t>(s.B) * static_cast<cuuint64_t>(s.H)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(s.D) * 2,
+                           static_cast<cuuint64_t>(s.S) * static_cast<cuuint64_t>(s.D) * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+xs_status check_shape(const xs_shape &s, bool need_ranks) {
+  if (s.B <= 0 || s.H <= 0 || s.S <= 0 || s.D <= 0 || s.P <= 0)
+    return fail(XS_ERR_INVALID_ARG, "non-positive size in shape B=%d H=%d S=%d D=%d P=%d", s.B, s.H,
+                s.S, s.D, s.P);
+  if (s.D % 8 != 0 || s.D > 128)
+    return fail(XS_ERR_UNSUPPORTED, "head dim D=%d unsupported (need D %% 8 == 0, 8 <= D <= 128)", s.D);
+  if (s.P > XS_MAX_RANKS)
+    return fail(XS_ERR_UNSUPPORTED, "P=%d exceeds XS_MAX_RANKS=%d", s.P, XS_MAX_RANKS);
+  if (need_ranks && (s.H % s.P != 0 || s.S % s.P != 0))
+    return fail(XS_ERR_UNSUPPORTED, "Ulysses sharding needs H %% P == 0 and S %% P == 0 (H=%d S=%d P=%d)",
+                s.H, s.S, s.P);
+  const long long elems = static_cast<long long>(s.B) * s.H * s.S * s.D;
+  if (elems <= 0 || elems > (1LL << 40))
+    return fail(XS_ERR_UNSUPPORTED, "tensor of %lld elements out of range", elems);
+  if (static_cast<long long>(s.B) * s.H * ((s.S + 255) / 256) > 0x7fffffffLL)
+    return fail(XS_ERR_UNSUPPORTED, "too many work items");
+  return XS_OK;
+}
+
+xs_status check_inputs(const void *q, const void *k, const void *v, const xs_shape &s) {
+  if (!q || !k || !v) return fail(XS_ERR_INVALID_ARG, "q, k and v must be non-null device pointers");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v))
+    return fail(XS_ERR_INVALID_ARG, "q, k and v must be 16-byte aligned");
+  (void)s;
+  return XS_OK;
+}
+
+xs_status check_dest(void *const *dest, const xs_shape &s, const void *const *inputs, int n_inputs) {
+  if (!dest) return fail(XS_ERR_INVALID_ARG, "dest must be a host array of P device pointers");
+  const uintptr_t slab = static_cast<uintptr_t>(s.B) * (s.S / s.P) * s.H * s.D * 2;
+  const uintptr_t full = static_cast<uintptr_t>(s.B) * s.H * s.S * s.D * 2;
+  for (int r = 0; r < s.P; ++r) {
+    if (!dest[r]) return fail(XS_ERR_INVALID_ARG, "dest[%d] is null", r);
+    if (!aligned16(dest[r])) return fail(XS_ERR_INVALID_ARG, "dest[%d] is not 16-byte aligned", r);
+    const Range a{reinterpret_cast<uintptr_t>(dest[r]), reinterpret_cast<uintptr_t>(dest[r]) + slab};
+    for (int o = 0; o < r; ++o) {
+      const Range b{reinterpret_cast<uintptr_t>(dest[o]), reinterpret_cast<uintptr_t>(dest[o]) + slab};
+      if (overlap(a, b)) return fail(XS_ERR_INVALID_ARG, "dest[%d] overlaps dest[%d]", r, o);
+    }
+    for (int i = 0; i < n_inputs; ++i) {
+      const Range b{reinterpret_cast<uintptr_t>(inputs[i]), reinterpret_cast<uintptr_t>(inputs[i]) + full};
+      if (overlap(a, b)) return fail(XS_ERR_INVALID_ARG, "dest[%d] overlaps an input tensor", r);
+    }
+  }
+  return XS_OK;
+}
+
+xs_status fill_attention(xs::AttnParams &p, const void *q, const void *k, const void *v,
+                         const xs_shape &s, float scale, int *dev_status) {
+  std::memset(&p, 0, sizeof(p));
+  if (!make_qkv_map(&p.tm_q, q, s) || !make_qkv_map(&p.tm_k, k, s) || !make_qkv_map(&p.tm_v, v, s))
+    return fail(XS_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point %s)",
+                encode_fn() ? "found" : "missing");
+  p.B = s.B;
+  p.H = s.H;
+  p.S = s.S;
+  p.D = s.D;
+  p.P = s.P;
+  p.S_local = s.S / s.P;
+  p.n_kv = (s.S + 127) / 128;
+  p.n_pairs = (s.S + 255) / 256;
+  p.n_items = s.B * s.H * p.n_pairs;
+  const double sc = scale > 0.f ? static_cast<double>(scale) : 1.0 / std::sqrt(static_cast<double>(s.D));
+  p.scale_log2 = static_cast<float>(sc * 1.4426950408889634);  // scale * log2(e)
+  p.status = dev_status;
+  p.wait_limit_ns = xs::kWaitLimitNs;
+  return XS_OK;
+}
+
+xs_status launched(cudaError_t e, const char *what) {
+  if (e != cudaSuccess) return fail(XS_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return ok();
+}
+
+}  // namespace
+
+namespace xs {
+int device_sm_count() {
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+}  // namespace xs
+
+extern "C" {
+
+xs_status xs_attn_a2a_fused(const void *q, const void *k, const void *v, void *const *dest,
+                            xs_shape shape, float scale, xs_stream_t stream, int *dev_status) {
+  xs_status st = check_shape(shape, true);
+  if (st != XS_OK) return st;
+  if ((st = check_inputs(q, k, v, shape)) != XS_OK) return st;
+  const void *ins[3] = {q, k, v};
+  if ((st = check_dest(dest, shape, ins, 3)) != XS_OK) return st;
+  xs::AttnParams p;
+  if ((st = fill_attention(p, q, k, v, shape, scale, dev_status)) != XS_OK) return st;
+  for (int r = 0; r < shape.P; ++r) p.dest[r] = dest[r];
+  return launched(xs::launch_attention(p, xs::kSeqScatter, reinterpret_cast<cudaStream_t>(stream)),
+                  "attention launch");
+}
+
+xs_status xs_attn(const void *q, const void *k, const void *v, void *out, xs_shape shape,
+                  float scale, xs_stream_t stream, int *dev_status) {
+  xs_status st = check_shape(shape, false);
+  if (st != XS_OK) return st;
+  if ((st = check_inputs(q, k, v, shape)) != XS_OK) return st;
+  if (!out || !aligned16(out)) return fail(XS_ERR_INVALID_ARG, "out must be a 16-byte aligned device pointer");
+  {
+    const uintptr_t full = static_cast<uintptr_t>(shape.B) * shape.H * shape.S * shape.D * 2;
+    const Range o{reinterpret_cast<uintptr_t>(out), reinterpret_cast<uintptr_t>(out) + full};
+    for (const void *in : {q, k, v}) {
+      const Range r{reinterpret_cast<uintptr_t>(in), reinterpret_cast<uintptr_t>(in) + full};
+      if (overlap(o, r)) return fail(XS_ERR_INVALID_ARG, "out overlaps an input tensor");
+    }
+  }
+  xs::AttnParams p;
+  if ((st = fill_attention(p, q, k, v, shape, scale, dev_status)) != XS_OK) return st;
+  p.out = out;
+  return launched(xs::launch_attention(p, xs::kHeadMajor, reinterpret_cast<cudaStream_t>(stream)),
+                  "attention launch");
+}
+
+xs_status xs_a2a_relayout(const void *src, void *const *dest, xs_shape shape, xs_stream_t stream) {
+  xs_status st = check_shape(shape, true);
+  if (st != XS_OK) return st;
+  if (!src || !aligned16(src)) return fail(XS_ERR_INVALID_ARG, "src must be a 16-byte aligned device pointer");
+  const void *ins[1] = {src};
+  if ((st = check_dest(dest, shape, ins, 1)) != XS_OK) return st;
+  xs::RelayoutParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.src = src;
+  for (int r = 0; r < shape.P; ++r) p.dest[r] = dest[r];
+  p.B = shape.B;
+  p.H = shape.H;
+  p.S = shape.S;
+  p.D = shape.D;
+  p.P = shape.P;
+  p.S_local = shape.S / shape.P;
+  return launched(xs::launch_relayout(p, reinterpret_cast<cudaStream_t>(stream)), "relayout launch");
+}
+
+xs_status xs_burst_probe(void *scratch, long long scratch_bytes, xs_burst_cfg cfg,
+                         unsigned long long *stamps, xs_stream_t stream) {
+  if (!scratch || !stamps || !aligned16(scratch) || (reinterpret_cast<uintptr_t>(stamps) & 7u))
+    return fail(XS_ERR_INVALID_ARG, "scratch (16-byte aligned) and stamps (8-byte aligned) are required");
+  if (cfg.producers < 1 || cfg.producers > 4096 || cfg.n_bursts < 1 || cfg.n_bursts > (1 << 20) ||
+      cfg.gap_cycles < 0 || cfg.gap_cycles > (1LL << 30) || cfg.burst_bytes <= 0 || scratch_bytes < 16 ||
+      cfg.threads_per_producer < 32 || cfg.threads_per_producer > 1024 || cfg.threads_per_producer % 32)
+    return fail(XS_ERR_INVALID_ARG, "burst probe configuration out of range");
+  if (cfg.burst_bytes % (16LL * cfg.producers) != 0)
+    return fail(XS_ERR_INVALID_ARG, "burst_bytes must be a multiple of 16 * producers");
+  const long long share = cfg.burst_bytes / 16 / cfg.producers;
+  if (share * cfg.producers > scratch_bytes / 16)
+    return fail(XS_ERR_INVALID_ARG, "one burst (%lld bytes) exceeds the scratch buffer", cfg.burst_bytes);
+  const Range a{reinterpret_cast<uintptr_t>(scratch), reinterpret_cast<uintptr_t>(scratch) + scratch_bytes};
+  const Range b{reinterpret_cast<uintptr_t>(stamps),
+                reinterpret_cast<uintptr_t>(stamps) + 32ull * cfg.producers * cfg.n_bursts};
+  if (overlap(a, b)) return fail(XS_ERR_INVALID_ARG, "stamps overlaps scratch");
+  xs::BurstParams p;
+  p.scratch = static_cast<uint4 *>(scratch);
+  p.scratch_chunks = scratch_bytes / 16;
+  p.share_chunks = share;
+  p.producers = cfg.producers;
+  p.n_bursts = cfg.n_bursts;
+  p.gap_iters = cfg.gap_cycles / 4;  // one dependent FMA is about 4 cycles
+  p.stamps = stamps;
+  return launched(xs::launch_burst_probe(p, cfg.threads_per_producer, reinterpret_cast<cudaStream_t>(stream)),
+                  "burst probe launch");
+}
+
+xs_status xs_selftest_bounded_wait(int *dev_status, long long limit_ns, xs_stream_t stream) {
+  if (!dev_status) return fail(XS_ERR_INVALID_ARG, "dev_status is required");
+  if (limit_ns < 1000 || limit_ns > 10000000000LL)
+    return fail(XS_ERR_INVALID_ARG, "limit_ns out of range [1e3, 1e10]");
+  return launched(xs::launch_wait_selftest(dev_status, limit_ns, reinterpret_cast<cudaStream_t>(stream)),
+                  "self-test launch");
+}
+
+const char *xs_get_error_string(xs_status status) {
+  switch (status) {
+    case XS_OK: return "XS_OK";
+    case XS_ERR_INVALID_ARG: return "XS_ERR_INVALID_ARG";
+    case XS_ERR_UNSUPPORTED: return "XS_ERR_UNSUPPORTED";
+    case XS_ERR_CUDA: return "XS_ERR_CUDA";
+    case XS_ERR_TIMEOUT: return "XS_ERR_TIMEOUT";
+  }
+  return "XS_ERR_UNKNOWN";
+}
+
+int xs_version(void) { return XS_VERSION; }
+
+const char *xs_last_error_detail(void) { return g_detail; }
+
+}  // extern "C"

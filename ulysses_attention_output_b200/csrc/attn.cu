@@ -1,0 +1,475 @@
+// attn.cu -- non-causal softmax attention on sm_100a with an epilogue that either writes the
+// head-major output or scatters each finished tile into the Ulysses sequence-shard slabs
+// (the post-attention All-to-All fused at tile granularity).
+//
+// Operation: O = softmax(Q K^T * scale) V per (b, h) -- page "X-Stage: An Overlooked
+// Pipeline Stage for Communication-Computation Overlap in DiT Inference", abstract and the
+// explainer's "Technisches Resuemee" -> "Zentrale Beitraege" -> "FlashAttention-A2A
+// (Piggybacking)": the owner of an output tile issues the stores of that tile into the
+// destination rank's sequence shard and immediately resumes the next tile's loop over keys,
+// which is the gap in which the issued stores drain.  No warp or SM is dedicated to the
+// exchange: the same warps that ran the softmax write the tile and go on.
+//
+// Structure of one persistent CTA (320 threads, one CTA per SM):
+//   warps 0-3  softmax for Q tile 0 (one thread per query row = one TMEM lane)
+//   warps 4-7  softmax for Q tile 1
+//   warp  8    TMA producer: Q tiles once per work item, then K_j, V_j through a 3-slot ring
+//   warp  9    TMEM allocator and single-thread tcgen05.mma issuer
+// A work item is 256 query rows (two 128-row tiles) of one (b, h).  Tensor memory holds
+//   cols [0,128)   S0 = Q0 K^T (fp32), overwritten in place by P0 (bf16 pairs, 64 cols)
+//   cols [128,256) S1 / P1
+//   cols [256,384) O0 (fp32, D padded to a multiple of 16)
+//   cols [384,512) O1
+// The MMA issue order per key tile j is QK0(j+1), PV1(j), QK1(j+1), PV0(j+1), so each tile's
+// softmax overlaps the other tile's two MMAs.  The running maximum is only moved when a new
+// row maximum exceeds it by more than 2^8 (in the exp2 domain); P then stays below 256 and
+// the rescale of O (done by the softmax thread itself, after the previous P V completed) is
+// rare.  P V consumes the probabilities rounded to bf16, and l sums those same rounded values
+// in fp32, so the normalised weights of every row add up to one.
+#include "xs_internal.cuh"
+
+namespace xs {
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kStages = 3;           // K/V ring slots
+constexpr int kChunkBytes = 16384;   // 128 rows x 128 bytes (64 bf16) per swizzle panel
+constexpr int kStageRows = 16;       // rows staged per warp per epilogue round
+constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest tolerated P before rescale
+
+// TMEM column of S_t / P_t and of O_t for Q tile t.
+__host__ __device__ constexpr uint32_t col_s(int t) { return 128u * static_cast<uint32_t>(t); }
+__host__ __device__ constexpr uint32_t col_o(int t) { return 256u + 128u * static_cast<uint32_t>(t); }
+
+// Shared memory layout (offsets from a 1024-byte aligned base).
+template <int DCH>
+struct Smem {
+  static constexpr uint32_t kTile = DCH * kChunkBytes;
+  static constexpr uint32_t kQ = 0;                                   // 2 tiles
+  static constexpr uint32_t kKV = kQ + 2 * kTile;                     // kStages tiles
+  static constexpr uint32_t kStage = kKV + kStages * kTile;           // 8 warps x 16 rows
+  static constexpr uint32_t kStageRowBytes = DCH * 128;
+  static constexpr uint32_t kStageBytes = 8 * kStageRows * kStageRowBytes;
+  static constexpr uint32_t kRowPtr = kStage + kStageBytes;           // 8 x 16 pointers
+  static constexpr uint32_t kBars = kRowPtr + 8 * kStageRows * 8;
+  // barriers: q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_done[2] drain
+  static constexpr uint32_t kNumBars = 2 + 2 + kStages + kStages + 2 + 2 + 2 + 1;
+  static constexpr uint32_t kMisc = kBars + kNumBars * 8;             // tmem base, abort flag
+  static constexpr uint32_t kTotal = kMisc + 16;
+  static constexpr size_t kAlloc = kTotal + 1024;                     // room for alignment
+};
+
+__device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
+
+template <int DCH, int EPI>
+__global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
+  using L = Smem<DCH>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = ptx::smem_u32(smem_raw);
+  const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
+  uint8_t *base = smem_raw + (base_u32 - raw_u32);
+
+  const uint32_t sQ = base_u32 + L::kQ;
+  const uint32_t sKV = base_u32 + L::kKV;
+  const uint32_t bar0 = base_u32 + L::kBars;
+  // barrier addresses
+  auto q_full = [&](int t) { return bar0 + 8u * (0 + t); };
+  auto q_empty = [&](int t) { return bar0 + 8u * (2 + t); };
+  auto kv_full = [&](uint32_t s) { return bar0 + 8u * (4 + s); };
+  auto kv_empty = [&](uint32_t s) { return bar0 + 8u * (4 + kStages + s); };
+  auto s_full = [&](int t) { return bar0 + 8u * (4 + 2 * kStages + t); };
+  auto p_full = [&](int t) { return bar0 + 8u * (6 + 2 * kStages + t); };
+  auto o_done = [&](int t) { return bar0 + 8u * (8 + 2 * kStages + t); };
+  const uint32_t drain_bar = bar0 + 8u * (10 + 2 * kStages);
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(base + L::kMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(base + L::kMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int t = 0; t < 2; ++t) {
+      ptx::mbar_init(q_full(t), 1);
+      ptx::mbar_init(q_empty(t), 1);
+      ptx::mbar_init(s_full(t), 1);
+      ptx::mbar_init(p_full(t), 128);
+      ptx::mbar_init(o_done(t), 1);
+    }
+    for (int s = 0; s < kStages; ++s) {
+      ptx::mbar_init(kv_full(s), 1);
+      ptx::mbar_init(kv_empty(s), 1);
+    }
+    ptx::mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 9) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_holder), 512);
+    ptx::tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    ptx::prefetch_tmap(&p.tm_q);
+    ptx::prefetch_tmap(&p.tm_k);
+    ptx::prefetch_tmap(&p.tm_v);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  const WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns};
+  const int n_kv = p.n_kv;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t kv_it = 0, it = 0;
+      int last_fill[kStages];
+      for (int s = 0; s < kStages; ++s) last_fill[s] = -1;
+      int q_filled[2] = {-1, -1};
+      bool ok = true;
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++it) {
+        const int bh = item / p.n_pairs;
+        const int q0 = (item - bh * p.n_pairs) * 256;
+        for (int t = 0; t < 2 && ok; ++t) {
+          ok = bounded_wait(q_empty(t), (it & 1u) ^ 1u, ctl);
+          if (!ok) break;
+          ptx::mbar_arrive_expect_tx(q_full(t), L::kTile);
+          for (int c = 0; c < DCH; ++c)
+            ptx::tma_load_3d(sQ + t * L::kTile + c * kChunkBytes, &p.tm_q, q_full(t), c * 64,
+                             q0 + 128 * t, bh);
+          q_filled[t] = static_cast<int>(it);
+        }
+        for (int j = 0; j < n_kv && ok; ++j) {
+          for (int kv = 0; kv < 2; ++kv) {
+            const uint32_t slot = kv_it % kStages;
+            ok = bounded_wait(kv_empty(slot), ((kv_it / kStages) & 1u) ^ 1u, ctl);
+            if (!ok) break;
+            ptx::mbar_arrive_expect_tx(kv_full(slot), L::kTile);
+            const CUtensorMap *tm = kv == 0 ? &p.tm_k : &p.tm_v;
+            for (int c = 0; c < DCH; ++c)
+              ptx::tma_load_3d(sKV + slot * L::kTile + c * kChunkBytes, tm, kv_full(slot), c * 64,
+                               j * 128, bh);
+            last_fill[slot] = static_cast<int>(kv_it);
+            ++kv_it;
+          }
+        }
+      }
+      if (!ok) {
+        // Abort: let every copy this thread started land before the CTA can exit.
+        for (int s = 0; s < kStages; ++s)
+          if (last_fill[s] >= 0)
+            bounded_wait_drain(kv_full(s), (static_cast<uint32_t>(last_fill[s]) / kStages) & 1u,
+                               p.wait_limit_ns);
+        for (int t = 0; t < 2; ++t)
+          if (q_filled[t] >= 0)
+            bounded_wait_drain(q_full(t), static_cast<uint32_t>(q_filled[t]) & 1u, p.wait_limit_ns);
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const int ks_qk = (p.D + 15) >> 4;             // K steps of 16 for Q K^T (true D)
+      const uint32_t n_pv = static_cast<uint32_t>(ks_qk * 16);  // N of P V (D padded to 16)
+      const uint32_t idesc_qk = ptx::idesc_bf16_f32(128, 128, 0);
+      const uint32_t idesc_pv = ptx::idesc_bf16_f32(128, n_pv, 1);
+      uint32_t kv_it = 0, it = 0, pc0 = 0, pc1 = 0;
+      bool ok = true;
+
+      auto issue_qk = [&](int t, uint32_t slot) {
+        const uint32_t a0 = sQ + t * L::kTile;
+        const uint32_t b0 = sKV + slot * L::kTile;
+        for (int ks = 0; ks < ks_qk; ++ks) {
+          const uint32_t off = (ks >> 2) * kChunkBytes + (ks & 3) * 32;
+          ptx::mma_ss(tmem + col_s(t), ptx::smem_desc_sw128(a0 + off, 16, 1024),
+                      ptx::smem_desc_sw128(b0 + off, 16, 1024), idesc_qk, ks > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, uint32_t slot, bool acc) {
+        const uint32_t b0 = sKV + slot * L::kTile;
+        for (int ks = 0; ks < 8; ++ks) {
+          // A = P (bf16 pairs in TMEM, 8 columns per 16 keys); B = V tile, MN-major:
+          // LBO = distance between 64-column panels, SBO = 8 key rows.
+          ptx::mma_ts(tmem + col_o(t), tmem + col_s(t) + ks * 8,
+                      ptx::smem_desc_sw128(b0 + ks * 2048, kChunkBytes, 1024), idesc_pv,
+                      (acc || ks > 0) ? 1u : 0u);
+        }
+      };
+
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++it) {
+        ok = bounded_wait(q_full(0), it & 1u, ctl) && bounded_wait(q_full(1), it & 1u, ctl);
+        if (!ok) break;
+        uint32_t slotK = kv_it % kStages;
+        ok = bounded_wait(kv_full(slotK), (kv_it / kStages) & 1u, ctl);
+        if (!ok) break;
+        ++kv_it;
+        ptx::tc_fence_after();
+        issue_qk(0, slotK);
+        ptx::mma_commit(s_full(0));
+        if (n_kv == 1) ptx::mma_commit(q_empty(0));
+        issue_qk(1, slotK);
+        ptx::mma_commit(s_full(1));
+        ptx::mma_commit(kv_empty(slotK));
+        if (n_kv == 1) ptx::mma_commit(q_empty(1));
+
+        for (int j = 0; j < n_kv && ok; ++j) {
+          const uint32_t slotV = kv_it % kStages;
+          ok = bounded_wait(kv_full(slotV), (kv_it / kStages) & 1u, ctl);
+          if (!ok) break;
+          ++kv_it;
+          ok = bounded_wait(p_full(0), pc0 & 1u, ctl);
+          if (!ok) break;
+          ++pc0;
+          ptx::tc_fence_after();
+          issue_pv(0, slotV, j > 0);
+          ptx::mma_commit(o_done(0));
+          const bool more = (j + 1) < n_kv;
+          if (more) {
+            slotK = kv_it % kStages;
+            ok = bounded_wait(kv_full(slotK), (kv_it / kStages) & 1u, ctl);
+            if (!ok) break;
+            ++kv_it;
+            ptx::tc_fence_after();
+            issue_qk(0, slotK);
+            ptx::mma_commit(s_full(0));
+            if (j + 2 == n_kv) ptx::mma_commit(q_empty(0));
+          }
+          ok = bounded_wait(p_full(1), pc1 & 1u, ctl);
+          if (!ok) break;
+          ++pc1;
+          ptx::tc_fence_after();
+          issue_pv(1, slotV, j > 0);
+          ptx::mma_commit(o_done(1));
+          ptx::mma_commit(kv_empty(slotV));
+          if (more) {
+            issue_qk(1, slotK);
+            ptx::mma_commit(s_full(1));
+            ptx::mma_commit(kv_empty(slotK));
+            if (j + 2 == n_kv) ptx::mma_commit(q_empty(1));
+          }
+        }
+      }
+      // Every MMA this thread issued must be complete before TMEM is released.
+      ptx::mma_commit(drain_bar);
+      bounded_wait_drain(drain_bar, 0, p.wait_limit_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int t = warp >> 2;         // Q tile of this warpgroup
+    const int wq = warp & 3;         // TMEM lane quadrant
+    const int row = wq * 32 + lane;  // query row within the tile
+    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_base + col_s(t);
+    const uint32_t tO = tmem + lane_base + col_o(t);
+    const float sl2 = p.scale_log2;
+    const int D = p.D;
+    const int nch = D >> 3;          // 16-byte chunks per output row
+    uint8_t *stg = base + L::kStage + warp * (kStageRows * L::kStageRowBytes);
+    uint8_t **rowptr = reinterpret_cast<uint8_t **>(base + L::kRowPtr) + warp * kStageRows;
+    uint32_t sc = 0;       // s_full phases consumed
+    uint32_t pv_base = 0;  // P V products of this tile completed before the current item
+    bool ok = true;
+
+    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      const int bh = item / p.n_pairs;
+      const int q0 = (item - bh * p.n_pairs) * 256;
+      float m_run = -INFINITY;  // running max in the exp2 domain (scaled)
+      float l_run = 0.f;
+
+      for (int j = 0; j < n_kv; ++j) {
+        ok = bounded_wait(s_full(t), sc & 1u, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ++sc;
+        ptx::tc_fence_after();
+        uint32_t sraw[128];
+        ptx::tmem_ld32(tS + 0, sraw + 0);
+        ptx::tmem_ld32(tS + 32, sraw + 32);
+        ptx::tmem_ld32(tS + 64, sraw + 64);
+        ptx::tmem_ld32(tS + 96, sraw + 96);
+        ptx::tmem_wait_ld();
+        float s[128];
+#pragma unroll
+        for (int c = 0; c < 128; ++c) s[c] = u2f(sraw[c]);
+        const int kv_valid = p.S - j * 128;
+        if (kv_valid < 128) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c >= kv_valid) s[c] = -INFINITY;
+        }
+        float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
+#pragma unroll
+        for (int c = 4; c < 128; c += 4) {
+          m0 = fmaxf(m0, s[c]);
+          m1 = fmaxf(m1, s[c + 1]);
+          m2 = fmaxf(m2, s[c + 2]);
+          m3 = fmaxf(m3, s[c + 3]);
+        }
+        const float mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * sl2;
+        bool rescale = false;
+        float alpha = 1.f;
+        if (mx > m_run + kRescaleThreshold) {
+          alpha = ptx::ex2(m_run - mx);  // 0 on the first tile (m_run = -inf)
+          l_run *= alpha;
+          m_run = mx;
+          rescale = (j > 0);
+        }
+        const float neg_m = -m_run;
+        float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+        uint32_t pk[64];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const float p0 = ptx::ex2(fmaf(s[2 * c + 0], sl2, neg_m));
+          const float p1 = ptx::ex2(fmaf(s[2 * c + 1], sl2, neg_m));
+          const float p2 = ptx::ex2(fmaf(s[2 * c + 2], sl2, neg_m));
+          const float p3 = ptx::ex2(fmaf(s[2 * c + 3], sl2, neg_m));
+          pk[c] = ptx::pack_bf16(p0, p1);
+          pk[c + 1] = ptx::pack_bf16(p2, p3);
+          // Row sum of the bf16-rounded probabilities, i.e. of exactly the weights P V uses.
+          l0 += u2f(pk[c] << 16);
+          l1 += u2f(pk[c] & 0xffff0000u);
+          l2 += u2f(pk[c + 1] << 16);
+          l3 += u2f(pk[c + 1] & 0xffff0000u);
+        }
+        l_run += (l0 + l1) + (l2 + l3);
+        ptx::tmem_st32(tS + 0, pk);
+        ptx::tmem_st32(tS + 32, pk + 32);
+        if (__any_sync(0xffffffffu, rescale)) {
+          // O holds P V of the previous key tiles: wait for the last of them, then scale.
+          ok = bounded_wait(o_done(t), (pv_base + j - 1) & 1u, ctl);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          const float a = rescale ? alpha : 1.f;
+#pragma unroll
+          for (int cc = 0; cc < DCH * 2; ++cc) {
+            uint32_t o[32];
+            ptx::tmem_ld32(tO + cc * 32, o);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(u2f(o[i]) * a);
+            ptx::tmem_st32(tO + cc * 32, o);
+          }
+        }
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(p_full(t));
+      }
+      if (!ok) break;
+
+      // ---------------------------------------------------------- epilogue
+      ok = bounded_wait(o_done(t), (pv_base + n_kv - 1) & 1u, ctl);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      pv_base += n_kv;
+      ptx::tc_fence_after();
+      const float inv_l = 1.f / l_run;
+      uint32_t ob[DCH * 32];
+#pragma unroll
+      for (int cc = 0; cc < DCH * 2; ++cc) {
+        uint32_t o[32];
+        ptx::tmem_ld32(tO + cc * 32, o);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          ob[cc * 16 + i] = ptx::pack_bf16(u2f(o[2 * i]) * inv_l, u2f(o[2 * i + 1]) * inv_l);
+      }
+      // Destination of this thread's row.
+      const int s_row = q0 + 128 * t + row;
+      uint8_t *dst_row = nullptr;
+      if (s_row < p.S) {
+        if constexpr (EPI == kHeadMajor) {
+          dst_row = static_cast<uint8_t *>(p.out) +
+                    (static_cast<size_t>(bh) * p.S + s_row) * static_cast<size_t>(D) * 2;
+        } else {
+          const int b = bh / p.H;
+          const int h = bh - b * p.H;
+          const int r = s_row / p.S_local;
+          const int sl = s_row - r * p.S_local;
+          dst_row = static_cast<uint8_t *>(p.dest[r]) +
+                    ((static_cast<size_t>(b) * p.S_local + sl) * p.H + h) * static_cast<size_t>(D) * 2;
+        }
+      }
+      // Two rounds of 16 rows per warp: stage rows in shared memory (chunk order rotated by
+      // row to spread banks), then write whole rows with consecutive lanes on consecutive
+      // 16-byte chunks.  The stores are not waited for: the warp goes straight on to its
+      // next tile while they drain.
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        if ((lane >> 4) == half) {
+          const int r16 = lane & 15;
+          const int rot = r16 % nch;
+          uint8_t *my = stg + r16 * L::kStageRowBytes;
+#pragma unroll
+          for (int c = 0; c < DCH * 8; ++c) {
+            if (c < nch) {
+              int pc = c + rot;
+              if (pc >= nch) pc -= nch;
+              *reinterpret_cast<uint4 *>(my + pc * 16) =
+                  make_uint4(ob[4 * c], ob[4 * c + 1], ob[4 * c + 2], ob[4 * c + 3]);
+            }
+          }
+          rowptr[r16] = dst_row;
+        }
+        __syncwarp();
+        for (int idx = lane; idx < kStageRows * nch; idx += 32) {
+          const int r16 = idx / nch;
+          const int c = idx - r16 * nch;
+          uint8_t *dr = rowptr[r16];
+          if (dr != nullptr) {
+            int pc = c + r16 % nch;
+            if (pc >= nch) pc -= nch;
+            const uint4 v = *reinterpret_cast<const uint4 *>(stg + r16 * L::kStageRowBytes + pc * 16);
+            ptx::st_global_v4(dr + c * 16, v);
+          }
+        }
+        __syncwarp();
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int DCH, int EPI>
+cudaError_t launch_impl(const AttnParams &p, cudaStream_t stream) {
+  using L = Smem<DCH>;
+  static_assert(L::kAlloc <= 232448, "shared memory budget exceeded");
+  auto kern = attn_fwd_kernel<DCH, EPI>;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static bool configured[64] = {};
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(L::kAlloc));
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  const int sms = device_sm_count();
+  if (sms <= 0) return cudaErrorInvalidDevice;
+  const int grid = p.n_items < sms ? p.n_items : sms;
+  kern<<<grid, kThreads, L::kAlloc, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t attention_smem_bytes(int dch) { return dch == 1 ? Smem<1>::kAlloc : Smem<2>::kAlloc; }
+
+cudaError_t launch_attention(const AttnParams &p, int epilogue, cudaStream_t stream) {
+  const int dch = p.D <= 64 ? 1 : 2;
+  if (dch == 1)
+    return epilogue == kHeadMajor ? launch_impl<1, kHeadMajor>(p, stream)
+                                  : launch_impl<1, kSeqScatter>(p, stream);
+  return epilogue == kHeadMajor ? launch_impl<2, kHeadMajor>(p, stream)
+                                : launch_impl<2, kSeqScatter>(p, stream);
+}
+
+}  // namespace xs

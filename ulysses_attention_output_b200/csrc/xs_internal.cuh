@@ -1,0 +1,104 @@
+// xs_internal.cuh -- types shared by the kernels and the C-ABI layer of libxs.so.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace xs {
+
+constexpr int kStatusOk = 0;
+constexpr int kStatusTimeout = 4;  // XS_ERR_TIMEOUT
+constexpr int kMaxRanks = 16;
+
+// Default bound of every on-device wait (global-timer nanoseconds).  A healthy wait in any
+// kernel here lasts microseconds; two seconds only ever trips when something is wrong.
+constexpr long long kWaitLimitNs = 2000000000LL;
+
+// Bounded wait on an mbarrier phase.  Returns false when the CTA-wide abort flag is set or
+// the limit passes; in the latter case it raises the abort flag and records XS_ERR_TIMEOUT
+// in *status (first error wins).  Never traps.
+struct WaitCtl {
+  volatile int *abort_flag;  // shared memory
+  int *status;               // device, nullable
+  long long limit_ns;
+};
+
+__device__ __forceinline__ void raise_timeout(const WaitCtl &c) {
+  *c.abort_flag = 1;
+  if (c.status) atomicCAS(c.status, kStatusOk, kStatusTimeout);
+}
+
+__device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, const WaitCtl &c) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  while (true) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*c.abort_flag) return false;
+    if (static_cast<long long>(ptx::globaltimer() - t0) > c.limit_ns) {
+      raise_timeout(c);
+      return false;
+    }
+  }
+}
+
+// Wait used only while shutting down after an abort: ignores the abort flag, still bounded.
+__device__ __forceinline__ bool bounded_wait_drain(uint32_t bar, uint32_t parity, long long limit_ns) {
+  const uint64_t t0 = ptx::globaltimer();
+  while (!ptx::mbar_try_wait(bar, parity)) {
+    if (static_cast<long long>(ptx::globaltimer() - t0) > limit_ns) return false;
+  }
+  return true;
+}
+
+// ---------------------------------------------------------------- attention
+enum EpilogueKind : int {
+  kHeadMajor = 0,   // out[b, h, s, :]
+  kSeqScatter = 1,  // dest[r][b, s_local, h, :]  (fused post-attention All-to-All)
+};
+
+struct AttnParams {
+  CUtensorMap tm_q;  // 3-D view {D, S, B*H} of q, box {64, 128, 1}, 128-byte swizzle
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  void *out;               // kHeadMajor
+  void *dest[kMaxRanks];   // kSeqScatter
+  int B, H, S, D, P;
+  int S_local;             // S / P
+  int n_kv;                // ceil(S / 128)
+  int n_pairs;             // ceil(S / 256): work items per (b, h)
+  int n_items;             // B * H * n_pairs
+  float scale_log2;        // softmax scale * log2(e)
+  int *status;
+  long long wait_limit_ns;
+};
+
+// Host launchers (attn.cu).
+cudaError_t launch_attention(const AttnParams &p, int epilogue, cudaStream_t stream);
+size_t attention_smem_bytes(int dch);
+
+// ---------------------------------------------------------------- exchange / probe
+struct RelayoutParams {
+  const void *src;
+  void *dest[kMaxRanks];
+  int B, H, S, D, P, S_local;
+};
+cudaError_t launch_relayout(const RelayoutParams &p, cudaStream_t stream);
+
+struct BurstParams {
+  uint4 *scratch;
+  long long scratch_chunks;  // 16-byte chunks in scratch
+  long long share_chunks;    // chunks per producer per burst
+  int producers;
+  int n_bursts;
+  long long gap_iters;       // dependent FMAs per thread after each burst
+  unsigned long long *stamps;
+};
+cudaError_t launch_burst_probe(const BurstParams &p, int threads, cudaStream_t stream);
+
+cudaError_t launch_wait_selftest(int *status, long long limit_ns, cudaStream_t stream);
+
+int device_sm_count();
+
+}  // namespace xs
