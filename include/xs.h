@@ -124,6 +124,32 @@ XS_API xs_status xs_burst_probe(void *scratch, long long scratch_bytes, xs_burst
                          unsigned long long *stamps, xs_stream_t stream);
 
 /*
+ * Allocation-free variant of xs_burst_probe.  (The pages have no counterpart: this exists for
+ * callers of this library, not for the method.)  Some callers cannot call cudaMalloc: a
+ * health-check or monitoring hook that runs inside a serving process whose device memory is
+ * already reserved by that process's caching allocator (an extra allocation can fail, or
+ * force the allocator to release and re-fragment its pool), or a runtime that forbids device
+ * allocation once it is initialised.  This entry point lets them run the probe with nothing
+ * but the stamps buffer they already own.
+ *   - Scratch: a fixed XS_BURST_STATIC_SCRATCH_BYTES (32 MiB) array in the library's own
+ *     global memory, held on every GPU that loads the library until the process exits.  The
+ *     bursts walk through it cyclically, so they stay L2-resident (32 MiB < L2); for
+ *     HBM-drain measurements use xs_burst_probe with a buffer larger than L2.
+ *   - burst_bytes above XS_BURST_STATIC_SCRATCH_BYTES is rejected with XS_ERR_UNSUPPORTED;
+ *     other limits and the stamps layout are those of xs_burst_probe.
+ *   - The first call on a device looks up the array's device address (once per device, with
+ *     that device current); make that first call before any stream capture.
+ *   - No cudaMalloc, cudaFree or allocating library routine is called.
+ *   - Every call shares the one array and leaves its contents behind; the probe only stores
+ *     into it, so nothing needs to start at zero.  Calls that overlap on the GPU (other
+ *     streams, other threads) race on the array: their stores interleave and each one's
+ *     stamps then include the other's traffic.
+ */
+#define XS_BURST_STATIC_SCRATCH_BYTES (32LL << 20)
+XS_API xs_status xs_burst_probe_static(xs_burst_cfg cfg, unsigned long long *stamps,
+                                       xs_stream_t stream);
+
+/*
  * Self-test of the bounded on-device wait used by every kernel in this library: launches
  * one thread that waits on a shared-memory barrier nothing ever arrives at, gives up after
  * limit_ns nanoseconds of global time (1e3 <= limit_ns <= 1e10) and writes XS_ERR_TIMEOUT

@@ -10,6 +10,7 @@ Calls (same names as the C ABI, without the ``xs_`` prefix):
 * :func:`attn`           -- attention with a head-major output.
 * :func:`a2a_relayout`   -- the exchange as a separate pass (serial baseline).
 * :func:`burst_probe`    -- Burst-Gap store microbenchmark.
+* :func:`burst_probe_static` -- the same, with no device allocation (fixed library scratch).
 * :func:`selftest_bounded_wait` -- exercises the bounded on-device wait.
 """
 from __future__ import annotations
@@ -21,7 +22,7 @@ import threading
 __all__ = [
     "XsError", "XS_OK", "XS_ERR_INVALID_ARG", "XS_ERR_UNSUPPORTED", "XS_ERR_CUDA", "XS_ERR_TIMEOUT",
     "library_path", "load", "version", "attn_a2a_fused", "attn", "a2a_relayout", "burst_probe",
-    "selftest_bounded_wait", "alloc_dest", "HostPipeline", "attention_flops",
+    "burst_probe_static", "selftest_bounded_wait", "alloc_dest", "HostPipeline", "attention_flops",
 ]
 
 XS_OK, XS_ERR_INVALID_ARG, XS_ERR_UNSUPPORTED, XS_ERR_CUDA, XS_ERR_TIMEOUT = 0, 1, 2, 3, 4
@@ -77,9 +78,10 @@ def load():
         lib.xs_attn.argtypes = [vp, vp, vp, vp, Shape, c_float, vp, ip]
         lib.xs_a2a_relayout.argtypes = [vp, vpp, Shape, vp]
         lib.xs_burst_probe.argtypes = [vp, ctypes.c_longlong, BurstCfg, vp, vp]
+        lib.xs_burst_probe_static.argtypes = [BurstCfg, vp, vp]
         lib.xs_selftest_bounded_wait.argtypes = [ip, ctypes.c_longlong, vp]
         for fn in (lib.xs_attn_a2a_fused, lib.xs_attn, lib.xs_a2a_relayout, lib.xs_burst_probe,
-                   lib.xs_selftest_bounded_wait):
+                   lib.xs_burst_probe_static, lib.xs_selftest_bounded_wait):
             fn.restype = c_int
         lib.xs_get_error_string.argtypes = [c_int]
         lib.xs_get_error_string.restype = ctypes.c_char_p
@@ -189,6 +191,19 @@ def burst_probe(scratch, stamps, burst_bytes: int, producers: int, gap_cycles: i
     nbytes = scratch.numel() * scratch.element_size()
     _check(load().xs_burst_probe(scratch.data_ptr(), nbytes, cfg, stamps.data_ptr(),
                                  _stream_handle(stream)))
+
+
+def burst_probe_static(stamps, burst_bytes: int, producers: int, gap_cycles: int, n_bursts: int,
+                       threads_per_producer: int = 256, stream=None):
+    """Burst-Gap microbenchmark that allocates nothing: the bursts go to the library's fixed
+    32 MiB scratch array instead of a caller buffer (see ``xs_burst_probe_static``)."""
+    import torch
+    if not stamps.is_cuda or stamps.dtype not in (torch.int64, torch.uint64) or \
+            stamps.numel() < producers * n_bursts * 4:
+        raise ValueError("stamps must be an int64/uint64 CUDA tensor with producers * n_bursts * 4 elements")
+    cfg = BurstCfg(int(burst_bytes), int(producers), int(gap_cycles), int(n_bursts),
+                   int(threads_per_producer))
+    _check(load().xs_burst_probe_static(cfg, stamps.data_ptr(), _stream_handle(stream)))
 
 
 def selftest_bounded_wait(status, limit_ns: int, stream=None):

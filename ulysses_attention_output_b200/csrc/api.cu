@@ -244,6 +244,36 @@ xs_status xs_burst_probe(void *scratch, long long scratch_bytes, xs_burst_cfg cf
                   "burst probe launch");
 }
 
+xs_status xs_burst_probe_static(xs_burst_cfg cfg, unsigned long long *stamps, xs_stream_t stream) {
+  if (!stamps || (reinterpret_cast<uintptr_t>(stamps) & 7u))
+    return fail(XS_ERR_INVALID_ARG, "stamps (8-byte aligned device pointer) is required");
+  if (cfg.producers < 1 || cfg.producers > 4096 || cfg.n_bursts < 1 || cfg.n_bursts > (1 << 20) ||
+      cfg.gap_cycles < 0 || cfg.gap_cycles > (1LL << 30) || cfg.burst_bytes <= 0 ||
+      cfg.threads_per_producer < 32 || cfg.threads_per_producer > 1024 || cfg.threads_per_producer % 32)
+    return fail(XS_ERR_INVALID_ARG, "burst probe configuration out of range");
+  if (cfg.burst_bytes % (16LL * cfg.producers) != 0)
+    return fail(XS_ERR_INVALID_ARG, "burst_bytes must be a multiple of 16 * producers");
+  if (cfg.burst_bytes > XS_BURST_STATIC_SCRATCH_BYTES)
+    return fail(XS_ERR_UNSUPPORTED,
+                "burst of %lld bytes exceeds the fixed %lld-byte scratch of xs_burst_probe_static; "
+                "use xs_burst_probe with a caller-allocated buffer",
+                cfg.burst_bytes, static_cast<long long>(XS_BURST_STATIC_SCRATCH_BYTES));
+  static_assert(XS_BURST_STATIC_SCRATCH_BYTES == xs::kStaticProbeScratchBytes, "scratch size mismatch");
+  uint4 *scratch = nullptr;
+  cudaError_t e = xs::static_probe_scratch(&scratch);
+  if (e != cudaSuccess) return fail(XS_ERR_CUDA, "scratch address lookup: %s", cudaGetErrorString(e));
+  xs::BurstParams p;
+  p.scratch = scratch;
+  p.scratch_chunks = XS_BURST_STATIC_SCRATCH_BYTES / 16;
+  p.share_chunks = cfg.burst_bytes / 16 / cfg.producers;
+  p.producers = cfg.producers;
+  p.n_bursts = cfg.n_bursts;
+  p.gap_iters = cfg.gap_cycles / 4;
+  p.stamps = stamps;
+  return launched(xs::launch_burst_probe(p, cfg.threads_per_producer, reinterpret_cast<cudaStream_t>(stream)),
+                  "burst probe launch");
+}
+
 xs_status xs_selftest_bounded_wait(int *dev_status, long long limit_ns, xs_stream_t stream) {
   if (!dev_status) return fail(XS_ERR_INVALID_ARG, "dev_status is required");
   if (limit_ns < 1000 || limit_ns > 10000000000LL)

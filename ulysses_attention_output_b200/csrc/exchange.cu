@@ -1,5 +1,7 @@
 // exchange.cu -- the stand-alone post-attention All-to-All (serial baseline), the Burst-Gap
 // store microbenchmark and the bounded-wait self-test.
+#include <mutex>
+
 #include "xs_internal.cuh"
 
 namespace xs {
@@ -106,6 +108,32 @@ __global__ void wait_selftest_kernel(int *status, long long limit_ns) {
 }
 
 }  // namespace
+
+// ---------------------------------------------------------------- fixed probe scratch
+// Scratch of the allocation-free probe entry point: a fixed array in the module's global
+// memory, reserved on every device that loads the library until the process exits.  Host
+// code must not pass `g_probe_scratch` itself to a kernel (on the host it names a host-side
+// stand-in); it uses the device address looked up once per device below.
+static __device__ __align__(256) uint4 g_probe_scratch[kStaticProbeScratchBytes / 16];
+
+cudaError_t static_probe_scratch(uint4 **out) {
+  static std::mutex mu;
+  static void *addr[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    // Once per device, with that device current.
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_probe_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *out = static_cast<uint4 *>(addr[dev]);
+  return cudaSuccess;
+}
 
 cudaError_t launch_relayout(const RelayoutParams &p, cudaStream_t stream) {
   const int sms = device_sm_count();

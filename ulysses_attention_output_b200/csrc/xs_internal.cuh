@@ -97,6 +97,11 @@ struct BurstParams {
 };
 cudaError_t launch_burst_probe(const BurstParams &p, int threads, cudaStream_t stream);
 
+// Allocation-free probe: device address of the fixed scratch array on the current device
+// (looked up on the first call per device), and its size.
+constexpr long long kStaticProbeScratchBytes = 32LL << 20;
+cudaError_t static_probe_scratch(uint4 **out);
+
 cudaError_t launch_wait_selftest(int *status, long long limit_ns, cudaStream_t stream);
 
 int device_sm_count();
