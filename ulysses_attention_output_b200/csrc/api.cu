@@ -9,7 +9,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/xs.h"
+#include "xs.h"
 #include "xs_internal.cuh"
 
 namespace {

@@ -25,7 +25,10 @@
 // row maximum exceeds it by more than 2^8 (in the exp2 domain); P then stays below 256 and
 // the rescale of O (done by the softmax thread itself, after the previous P V completed) is
 // rare.  P V consumes the probabilities rounded to bf16, and l sums those same rounded values
-// in fp32, so the normalised weights of every row add up to one.
+// in fp32, so the normalised weights of every row add up to one.  The softmax works on column
+// pairs in packed fp32 (f32x2) and computes 5 of every 16 pairs of exponentials with an FMA-pipe
+// polynomial instead of MUFU ex2, because at one exponential per 4*D FLOPs MUFU alone would
+// take as long as the tensor core.
 #include "xs_internal.cuh"
 
 namespace xs {
@@ -60,6 +63,40 @@ struct Smem {
 };
 
 __device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
+__device__ __forceinline__ uint32_t f2u(float x) { return __float_as_uint(x); }
+
+// Column pairs (of 64 per 128-key tile) whose exponentials run on the FMA pipe instead of
+// MUFU: kEmulatedPer16 of every 16 pairs, spread evenly.
+#ifndef XS_EMULATED_PER16
+#define XS_EMULATED_PER16 5
+#endif
+constexpr int kEmulatedPer16 = XS_EMULATED_PER16;
+__host__ __device__ constexpr bool emulated_pair(int c) {
+  return ((c * kEmulatedPer16) & 15) < kEmulatedPer16;
+}
+
+// 2^x for a pair of fp32 values on the FMA pipe (no MUFU).  Range reduction x = n + f with
+// n = round-to-nearest(x) obtained by adding and subtracting 1.5 * 2^23, f in [-1/2, 1/2];
+// 2^f by a degree-3 polynomial with p(0) = 1 fitted for minimax relative error (1.0e-4) by
+// csrc/fit_exp2_poly.py; 2^n applied by adding n to the exponent field.  Inputs below -127
+// are clamped there, which yields exactly +0; masked entries (-inf) therefore give 0.
+__device__ __forceinline__ void exp2_fma_pair(uint64_t x2, float &p0, float &p1) {
+  constexpr uint32_t kC1 = 0x3f317afdu, kC2 = 0x3e780627u, kC3 = 0x3d61512eu;
+  float x0, x1;
+  ptx::f2x_split(x2, x0, x1);
+  const uint64_t x = ptx::f2x(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+  const uint64_t shifter = ptx::f2x(12582912.f, 12582912.f);
+  const uint64_t t = ptx::add2(x, shifter);
+  const uint64_t f = ptx::sub2(x, ptx::sub2(t, shifter));
+  uint64_t q = ptx::fma2(f, ptx::f2x(u2f(kC3), u2f(kC3)), ptx::f2x(u2f(kC2), u2f(kC2)));
+  q = ptx::fma2(q, f, ptx::f2x(u2f(kC1), u2f(kC1)));
+  q = ptx::fma2(q, f, ptx::f2x(1.f, 1.f));
+  float q0, q1, t0, t1;
+  ptx::f2x_split(q, q0, q1);
+  ptx::f2x_split(t, t0, t1);
+  p0 = u2f(f2u(q0) + (f2u(t0) << 23));
+  p1 = u2f(f2u(q1) + (f2u(t1) << 23));
+}
 
 template <int DCH, int EPI>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
@@ -92,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       ptx::mbar_init(q_full(t), 1);
       ptx::mbar_init(q_empty(t), 1);
       ptx::mbar_init(s_full(t), 1);
-      ptx::mbar_init(p_full(t), 128);
+      ptx::mbar_init(p_full(t), 4);  // one arrival per softmax warp
       ptx::mbar_init(o_done(t), 1);
     }
     for (int s = 0; s < kStages; ++s) {
@@ -124,9 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t kv_it = 0, it = 0;
-      int last_fill[kStages];
-      for (int s = 0; s < kStages; ++s) last_fill[s] = -1;
-      int q_filled[2] = {-1, -1};
+      int q_filled0 = -1, q_filled1 = -1;
       bool ok = true;
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++it) {
         const int bh = item / p.n_pairs;
@@ -138,7 +173,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           for (int c = 0; c < DCH; ++c)
             ptx::tma_load_3d(sQ + t * L::kTile + c * kChunkBytes, &p.tm_q, q_full(t), c * 64,
                              q0 + 128 * t, bh);
-          q_filled[t] = static_cast<int>(it);
+          if (t == 0) q_filled0 = static_cast<int>(it);
+          else q_filled1 = static_cast<int>(it);
         }
         for (int j = 0; j < n_kv && ok; ++j) {
           for (int kv = 0; kv < 2; ++kv) {
@@ -150,20 +186,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             for (int c = 0; c < DCH; ++c)
               ptx::tma_load_3d(sKV + slot * L::kTile + c * kChunkBytes, tm, kv_full(slot), c * 64,
                                j * 128, bh);
-            last_fill[slot] = static_cast<int>(kv_it);
             ++kv_it;
           }
         }
       }
       if (!ok) {
         // Abort: let every copy this thread started land before the CTA can exit.
-        for (int s = 0; s < kStages; ++s)
-          if (last_fill[s] >= 0)
-            bounded_wait_drain(kv_full(s), (static_cast<uint32_t>(last_fill[s]) / kStages) & 1u,
-                               p.wait_limit_ns);
-        for (int t = 0; t < 2; ++t)
-          if (q_filled[t] >= 0)
-            bounded_wait_drain(q_full(t), static_cast<uint32_t>(q_filled[t]) & 1u, p.wait_limit_ns);
+        // The ring slots hold the last (up to) kStages fills, numbered kv_it - kStages .. kv_it - 1.
+        for (uint32_t f = kv_it > kStages ? kv_it - kStages : 0; f < kv_it; ++f)
+          bounded_wait_drain(kv_full(f % kStages), (f / kStages) & 1u, p.wait_limit_ns);
+        if (q_filled0 >= 0)
+          bounded_wait_drain(q_full(0), static_cast<uint32_t>(q_filled0) & 1u, p.wait_limit_ns);
+        if (q_filled1 >= 0)
+          bounded_wait_drain(q_full(1), static_cast<uint32_t>(q_filled1) & 1u, p.wait_limit_ns);
       }
     }
   } else if (warp == 9) {
@@ -176,22 +211,33 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       uint32_t kv_it = 0, it = 0, pc0 = 0, pc1 = 0;
       bool ok = true;
 
+      // Descriptors are built once; per MMA only compile-time offsets are added (a per-MMA
+      // rebuild in the issue loop costs ~1.5x the MMA time of a 128x128x16 step).  Adding to
+      // the start-address field never carries: shared addresses are below 2^18 bytes.
+      const uint64_t dq0 = ptx::smem_desc_sw128(sQ, 16, 1024);
+      const uint64_t dk0 = ptx::smem_desc_sw128(sKV, 16, 1024);
+      const uint64_t dv0 = ptx::smem_desc_sw128(sKV, kChunkBytes, 1024);
+      constexpr uint64_t kTileDesc = L::kTile >> 4;  // one tile, in descriptor address units
+
       auto issue_qk = [&](int t, uint32_t slot) {
-        const uint32_t a0 = sQ + t * L::kTile;
-        const uint32_t b0 = sKV + slot * L::kTile;
-        for (int ks = 0; ks < ks_qk; ++ks) {
-          const uint32_t off = (ks >> 2) * kChunkBytes + (ks & 3) * 32;
-          ptx::mma_ss(tmem + col_s(t), ptx::smem_desc_sw128(a0 + off, 16, 1024),
-                      ptx::smem_desc_sw128(b0 + off, 16, 1024), idesc_qk, ks > 0 ? 1u : 0u);
+        const uint64_t a = dq0 + static_cast<uint64_t>(t) * kTileDesc;
+        const uint64_t b = dk0 + static_cast<uint64_t>(slot) * kTileDesc;
+        const uint32_t d = tmem + col_s(t);
+#pragma unroll
+        for (int ks = 0; ks < DCH * 4; ++ks) {
+          const uint64_t off = static_cast<uint64_t>(((ks >> 2) * kChunkBytes + (ks & 3) * 32) >> 4);
+          if (ks < ks_qk) ptx::mma_ss(d, a + off, b + off, idesc_qk, ks > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, uint32_t slot, bool acc) {
-        const uint32_t b0 = sKV + slot * L::kTile;
+        const uint64_t b = dv0 + static_cast<uint64_t>(slot) * kTileDesc;
+        const uint32_t d = tmem + col_o(t);
+        const uint32_t a = tmem + col_s(t);
+#pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           // A = P (bf16 pairs in TMEM, 8 columns per 16 keys); B = V tile, MN-major:
           // LBO = distance between 64-column panels, SBO = 8 key rows.
-          ptx::mma_ts(tmem + col_o(t), tmem + col_s(t) + ks * 8,
-                      ptx::smem_desc_sw128(b0 + ks * 2048, kChunkBytes, 1024), idesc_pv,
+          ptx::mma_ts(d, a + ks * 8, b + static_cast<uint64_t>(ks * (2048 >> 4)), idesc_pv,
                       (acc || ks > 0) ? 1u : 0u);
         }
       };
@@ -282,30 +328,36 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         if (!ok) break;
         ++sc;
         ptx::tc_fence_after();
-        uint32_t sraw[128];
-        ptx::tmem_ld32(tS + 0, sraw + 0);
-        ptx::tmem_ld32(tS + 32, sraw + 32);
-        ptx::tmem_ld32(tS + 64, sraw + 64);
-        ptx::tmem_ld32(tS + 96, sraw + 96);
-        ptx::tmem_wait_ld();
-        float s[128];
+        const int kv_valid = p.S - j * 128;  // < 128 only on a ragged last key tile
+        // Pass 1: row maximum over the 128 scores (one TMEM round trip for the whole row).
+        float m0, m1, m2, m3;
+        {
+          uint32_t sr[128];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] = u2f(sraw[c]);
-        const int kv_valid = p.S - j * 128;
-        if (kv_valid < 128) {
+          for (int q = 0; q < 4; ++q) ptx::tmem_ld32(tS + 32 * q, sr + 32 * q);
+          ptx::tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c >= kv_valid) s[c] = -INFINITY;
+          for (int q = 0; q < 4; ++q) ptx::reg_fence32(sr + 32 * q);
+          if (kv_valid < 128) {
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+              if (c >= kv_valid) sr[c] = 0xff800000u;  // -inf
+          }
+          m0 = u2f(sr[0]);
+          m1 = u2f(sr[1]);
+          m2 = u2f(sr[2]);
+          m3 = u2f(sr[3]);
+#pragma unroll
+          for (int c = 4; c < 124; c += 8) {
+            m0 = ptx::max3(m0, u2f(sr[c]), u2f(sr[c + 1]));
+            m1 = ptx::max3(m1, u2f(sr[c + 2]), u2f(sr[c + 3]));
+            m2 = ptx::max3(m2, u2f(sr[c + 4]), u2f(sr[c + 5]));
+            m3 = ptx::max3(m3, u2f(sr[c + 6]), u2f(sr[c + 7]));
+          }
+          m0 = ptx::max3(m0, u2f(sr[124]), u2f(sr[125]));
+          m1 = ptx::max3(m1, u2f(sr[126]), u2f(sr[127]));
         }
-        float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
-#pragma unroll
-        for (int c = 4; c < 128; c += 4) {
-          m0 = fmaxf(m0, s[c]);
-          m1 = fmaxf(m1, s[c + 1]);
-          m2 = fmaxf(m2, s[c + 2]);
-          m3 = fmaxf(m3, s[c + 3]);
-        }
-        const float mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * sl2;
+        const float mx = ptx::max3(m0, m1, fmaxf(m2, m3)) * sl2;
         bool rescale = false;
         float alpha = 1.f;
         if (mx > m_run + kRescaleThreshold) {
@@ -314,26 +366,66 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           m_run = mx;
           rescale = (j > 0);
         }
-        const float neg_m = -m_run;
-        float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
-        uint32_t pk[64];
+        // Pass 2, 32 columns at a time: p = 2^(s * scale * log2 e - m) in packed fp32 pairs,
+        // rounded to bf16 pairs and stored over the already-consumed S columns as P (the P
+        // words of chunk c land in columns [16c, 16c+16), which pass 2 has read already).
+        // A fixed subset of the pairs uses the FMA-pipe exponential instead of MUFU.
+        const uint64_t sl2x2 = ptx::f2x(sl2, sl2);
+        const uint64_t negm2 = ptx::f2x(-m_run, -m_run);
+        uint64_t lacc0 = 0, lacc1 = 0;  // packed row sums (0 bits == +0.0f)
+        auto exp_chunk = [&](int ch, uint32_t(&sr)[32]) {
+          if (kv_valid < 128) {
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float p0 = ptx::ex2(fmaf(s[2 * c + 0], sl2, neg_m));
-          const float p1 = ptx::ex2(fmaf(s[2 * c + 1], sl2, neg_m));
-          const float p2 = ptx::ex2(fmaf(s[2 * c + 2], sl2, neg_m));
-          const float p3 = ptx::ex2(fmaf(s[2 * c + 3], sl2, neg_m));
-          pk[c] = ptx::pack_bf16(p0, p1);
-          pk[c + 1] = ptx::pack_bf16(p2, p3);
-          // Row sum of the bf16-rounded probabilities, i.e. of exactly the weights P V uses.
-          l0 += u2f(pk[c] << 16);
-          l1 += u2f(pk[c] & 0xffff0000u);
-          l2 += u2f(pk[c + 1] << 16);
-          l3 += u2f(pk[c + 1] & 0xffff0000u);
+            for (int c = 0; c < 32; ++c)
+              if (32 * ch + c >= kv_valid) sr[c] = 0xff800000u;
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const uint64_t x2 = ptx::fma2(ptx::f2x(u2f(sr[2 * c]), u2f(sr[2 * c + 1])), sl2x2, negm2);
+            float p0, p1;
+            if (emulated_pair(16 * ch + c)) {
+              exp2_fma_pair(x2, p0, p1);
+            } else {
+              float x0, x1;
+              ptx::f2x_split(x2, x0, x1);
+              p0 = ptx::ex2(x0);
+              p1 = ptx::ex2(x1);
+            }
+            pk[c] = ptx::pack_bf16(p0, p1);
+            // Row sum of the bf16-rounded probabilities, i.e. of exactly the weights P V uses.
+            const uint64_t r2 = ptx::f2x(u2f(pk[c] << 16), u2f(pk[c] & 0xffff0000u));
+            if (c & 1)
+              lacc1 = ptx::add2(lacc1, r2);
+            else
+              lacc0 = ptx::add2(lacc0, r2);
+          }
+          ptx::tmem_st16(tS + 16 * ch, pk);
+        };
+        // Two register buffers: the load of chunk c+1 is in flight while chunk c is computed.
+        uint32_t buf0[32], buf1[32];
+        ptx::tmem_ld32(tS + 0, buf0);
+        ptx::tmem_wait_ld();
+        ptx::reg_fence32(buf0);
+        ptx::tmem_ld32(tS + 32, buf1);
+        exp_chunk(0, buf0);
+        ptx::tmem_wait_ld();
+        ptx::reg_fence32(buf1);
+        ptx::tmem_ld32(tS + 64, buf0);
+        exp_chunk(1, buf1);
+        ptx::tmem_wait_ld();
+        ptx::reg_fence32(buf0);
+        ptx::tmem_ld32(tS + 96, buf1);
+        exp_chunk(2, buf0);
+        ptx::tmem_wait_ld();
+        ptx::reg_fence32(buf1);
+        exp_chunk(3, buf1);
+        {
+          float a0, a1, b0, b1;
+          ptx::f2x_split(lacc0, a0, a1);
+          ptx::f2x_split(lacc1, b0, b1);
+          l_run += (a0 + a1) + (b0 + b1);
         }
-        l_run += (l0 + l1) + (l2 + l3);
-        ptx::tmem_st32(tS + 0, pk);
-        ptx::tmem_st32(tS + 32, pk + 32);
         if (__any_sync(0xffffffffu, rescale)) {
           // O holds P V of the previous key tiles: wait for the last of them, then scale.
           ok = bounded_wait(o_done(t), (pv_base + j - 1) & 1u, ctl);
@@ -346,6 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             uint32_t o[32];
             ptx::tmem_ld32(tO + cc * 32, o);
             ptx::tmem_wait_ld();
+            ptx::reg_fence32(o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(u2f(o[i]) * a);
             ptx::tmem_st32(tO + cc * 32, o);
@@ -353,7 +446,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         }
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
-        ptx::mbar_arrive(p_full(t));
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(p_full(t));  // one arrival per warp
       }
       if (!ok) break;
 
@@ -364,16 +458,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       pv_base += n_kv;
       ptx::tc_fence_after();
       const float inv_l = 1.f / l_run;
-      uint32_t ob[DCH * 32];
-#pragma unroll
-      for (int cc = 0; cc < DCH * 2; ++cc) {
-        uint32_t o[32];
-        ptx::tmem_ld32(tO + cc * 32, o);
-        ptx::tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          ob[cc * 16 + i] = ptx::pack_bf16(u2f(o[2 * i]) * inv_l, u2f(o[2 * i + 1]) * inv_l);
-      }
       // Destination of this thread's row.
       const int s_row = q0 + 128 * t + row;
       uint8_t *dst_row = nullptr;
@@ -394,23 +478,37 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       // row to spread banks), then write whole rows with consecutive lanes on consecutive
       // 16-byte chunks.  The stores are not waited for: the warp goes straight on to its
       // next tile while they drain.
+      // O is read from TMEM once per round, 32 columns at a time (the warp-collective load
+      // brings all 32 rows; the lanes of the current round keep theirs).
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        if ((lane >> 4) == half) {
-          const int r16 = lane & 15;
-          const int rot = r16 % nch;
-          uint8_t *my = stg + r16 * L::kStageRowBytes;
+        const bool mine = (lane >> 4) == half;
+        const int r16 = lane & 15;
+        const int rot = r16 % nch;
+        uint8_t *my = stg + r16 * L::kStageRowBytes;
 #pragma unroll
-          for (int c = 0; c < DCH * 8; ++c) {
-            if (c < nch) {
-              int pc = c + rot;
-              if (pc >= nch) pc -= nch;
-              *reinterpret_cast<uint4 *>(my + pc * 16) =
-                  make_uint4(ob[4 * c], ob[4 * c + 1], ob[4 * c + 2], ob[4 * c + 3]);
+        for (int cc = 0; cc < DCH * 2; ++cc) {
+          uint32_t o[32];
+          ptx::tmem_ld32(tO + cc * 32, o);
+          ptx::tmem_wait_ld();
+          ptx::reg_fence32(o);
+          if (mine) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const int c = cc * 4 + q4;  // 16-byte chunk (8 columns) of the output row
+              if (c < nch) {
+                int pc = c + rot;
+                if (pc >= nch) pc -= nch;
+                uint32_t w[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                  w[i] = ptx::pack_bf16(u2f(o[8 * q4 + 2 * i]) * inv_l, u2f(o[8 * q4 + 2 * i + 1]) * inv_l);
+                *reinterpret_cast<uint4 *>(my + pc * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+              }
             }
           }
-          rowptr[r16] = dst_row;
         }
+        if (mine) rowptr[r16] = dst_row;
         __syncwarp();
         for (int idx = lane; idx < kStageRows * nch; idx += 32) {
           const int r16 = idx / nch;

@@ -30,11 +30,15 @@ __device__ __forceinline__ void raise_timeout(const WaitCtl &c) {
   if (c.status) atomicCAS(c.status, kStatusOk, kStatusTimeout);
 }
 
+#ifndef XS_WAIT_SLEEP_NS
+#define XS_WAIT_SLEEP_NS 20000
+#endif
+
 __device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, const WaitCtl &c) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer();
   while (true) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (ptx::mbar_try_wait_sleep(bar, parity, XS_WAIT_SLEEP_NS)) return true;
     if (*c.abort_flag) return false;
     if (static_cast<long long>(ptx::globaltimer() - t0) > c.limit_ns) {
       raise_timeout(c);
