@@ -1,0 +1,224 @@
+"""Burst-Gap characterisation of store bursts on one B200.
+
+The Burst-Gap model of the X-Stage paper (explainer page, "Technisches Resuemee" ->
+"Methodik: Die X-Stage-Abstraktion und das Burst-Gap-Modell") gives the sender-visible issue
+time of a burst of aggregate volume V issued by K producers that compute for a gap G between
+bursts as
+
+    T_iss(G; K, V) = max(T0_iss(K, V), V / R - G)
+
+with T0_iss the backpressure-free issue time, R the effective drain rate and Q the effective
+outstanding capacity (the volume that can be in flight before issue stalls).  The pages give
+the model and its parameters by name only (R of about 717 GB/s on their remote-store path; no
+T0_iss or Q values).
+
+This module measures T_iss with the ``xs_burst_probe`` kernel (16-byte stores into a scratch
+ring in this GPU's memory, i.e. the local stand-in for remote stores) over a grid of
+(K, V, G), and fits the three parameters:
+
+* T0_iss(K, V): the issue time at the largest gaps, where every earlier burst has drained;
+* R: 1 / slope of T_iss against V at G = 0 over the volumes in the drain-dominated regime
+  (issue time more than 25% above the backpressure-free time);
+* Q: the knee -- the largest volume at G = 0 whose issue time is still within 25% of the
+  backpressure-free time at that volume.
+
+``predict`` evaluates the model; ``completion_coupled`` is the counter-model in which the
+issuer waits until its stores have drained (issue time V / R for every burst, no overlap).
+
+Run ``python -m ulysses_attention_output_b200.burst_gap [--large] [--wide] [--fused]`` on a GPU
+for a sweep (``--large``: bursts of 4..64 MB from 148 producers; ``--wide``: 1024 threads per
+producer; ``--fused``: also time the fused kernel against attention alone on the MMDiT, long
+and video workloads and set the measured overhead beside both models' predictions); it
+prints one JSON object with the raw points and the fit.
+"""
+from __future__ import annotations
+
+import json
+import math
+import sys
+
+import numpy as np
+
+
+# ----------------------------------------------------------------------------- model
+def predict(t0_ns: float, r_gbs: float, volume_bytes: float, gap_ns: float) -> float:
+    """Burst-Gap model: sender-visible issue time (ns) of one burst."""
+    return max(t0_ns, volume_bytes / r_gbs - gap_ns)
+
+
+def completion_coupled(r_gbs: float, volume_bytes: float) -> float:
+    """Counter-model: the issuer waits for its burst to drain before it resumes (ns)."""
+    return volume_bytes / r_gbs
+
+
+# ----------------------------------------------------------------------------- measurement
+def issue_times_ns(stamps: np.ndarray, drop: int = 8):
+    """Per-burst sender-visible issue times (ns) from the probe's stamps [K, N, 4].
+
+    Cycles are converted with the SM clock rate measured from the same stamps (clock64 and
+    global-timer deltas between the first kept burst and the last one of each producer).
+    Returns (issue_ns [K, N-drop], gap_ns [K, N-drop], clock_ghz).
+    """
+    st = np.asarray(stamps, dtype=np.int64)
+    k, n, _ = st.shape
+    if n - drop < 2:
+        raise ValueError("need at least two bursts after the dropped ones")
+    kept = st[:, drop:, :]
+    d_clk = (kept[:, -1, 0] - kept[:, 0, 0]).astype(np.float64)
+    d_ns = (kept[:, -1, 3] - kept[:, 0, 3]).astype(np.float64)
+    ok = d_ns > 0
+    ghz = float(np.median(d_clk[ok] / d_ns[ok])) if ok.any() else float("nan")
+    issue = (kept[:, :, 1] - kept[:, :, 0]) / ghz
+    gap = (kept[:, :, 2] - kept[:, :, 1]) / ghz
+    return issue, gap, ghz
+
+
+def run_point(xs, torch, scratch, producers: int, volume: int, gap_cycles: int, n_bursts: int,
+              threads: int = 256, drop: int = 8):
+    stamps = torch.zeros((producers, n_bursts, 4), dtype=torch.int64, device=scratch.device)
+    xs.burst_probe(scratch, stamps, burst_bytes=volume, producers=producers, gap_cycles=gap_cycles,
+                   n_bursts=n_bursts, threads_per_producer=threads)
+    torch.cuda.synchronize()
+    issue, gap, ghz = issue_times_ns(stamps.cpu().numpy(), drop)
+    return {"K": producers, "V": volume, "G_cycles": gap_cycles, "G_ns": float(np.median(gap)),
+            "t_iss_ns": float(np.median(issue)), "t_iss_p90_ns": float(np.percentile(issue, 90)),
+            "clock_ghz": ghz}
+
+
+def sweep(volumes, producers, gaps, n_bursts: int = 64, drop: int = 8,
+          scratch_bytes: int = 1 << 30, threads: int = 256):
+    """Measure T_iss over the (K, V, G) grid.  Volumes are per burst over all producers."""
+    import torch
+
+    import ulysses_attention_output_b200 as xs
+    scratch = torch.empty(scratch_bytes, dtype=torch.uint8, device="cuda")
+    out = []
+    for k in producers:
+        for v in volumes:
+            vv = (v // (16 * k)) * 16 * k
+            if vv <= 0:
+                continue
+            for g in gaps:
+                out.append(run_point(xs, torch, scratch, k, vv, g, n_bursts, threads, drop))
+    return out
+
+
+# ----------------------------------------------------------------------------- fit
+def fit(points, knee_tolerance: float = 0.25):
+    """Fit T0_iss(K, V), R and Q from sweep points (dicts with K, V, G_ns, t_iss_ns)."""
+    by_kv = {}
+    for p in points:
+        by_kv.setdefault((p["K"], p["V"]), []).append(p)
+    t0 = {}
+    for (k, v), pts in by_kv.items():
+        gmax = max(q["G_ns"] for q in pts)
+        floor = [q["t_iss_ns"] for q in pts if q["G_ns"] >= 0.5 * gmax]
+        t0[(k, v)] = float(min(floor))
+    kmax = max(k for k, _ in by_kv)
+    zero_gap = sorted(((v, min(q["t_iss_ns"] for q in pts if q["G_ns"] == min(x["G_ns"] for x in pts)))
+                       for (k, v), pts in by_kv.items() if k == kmax))
+    vols = np.array([v for v, _ in zero_gap], dtype=np.float64)
+    times = np.array([t for _, t in zero_gap], dtype=np.float64)
+    knee = None
+    for v, t in zero_gap:
+        if t <= (1.0 + knee_tolerance) * t0[(kmax, int(v))]:
+            knee = int(v)
+    # drain-dominated points: issue time at G = 0 clearly above the backpressure-free time
+    drain = np.array([t > (1.0 + knee_tolerance) * t0[(kmax, int(v))] for v, t in zero_gap])
+    if drain.sum() < 2:
+        drain = vols >= np.sort(vols)[-3]
+    slope, intercept = np.polyfit(vols[drain], times[drain], 1)
+    r_gbs = 1.0 / slope if slope > 0 else float("inf")
+    return {"T0_ns": {f"K={k},V={v}": val for (k, v), val in sorted(t0.items())},
+            "R_GBps": float(r_gbs), "intercept_ns": float(intercept), "Q_bytes": knee,
+            "K_for_R": kmax}
+
+
+def t0_at(points, k: int, volume: float) -> float:
+    """Backpressure-free issue time at (k, volume), linear in V between / beyond the two
+    nearest swept volumes of the largest gaps."""
+    f = fit([p for p in points if p["K"] == k])
+    vols = sorted(int(key.split("V=")[1]) for key in f["T0_ns"])
+    t = [f["T0_ns"][f"K={k},V={v}"] for v in vols]
+    if volume <= vols[0]:
+        return t[0]
+    i = max(j for j in range(len(vols) - 1) if vols[j] <= volume) if volume < vols[-1] else len(vols) - 2
+    return t[i] + (t[i + 1] - t[i]) * (volume - vols[i]) / (vols[i + 1] - vols[i])
+
+
+def epilogue_models(points, n_ctas: int, bytes_per_cta: int, gap_ns: float):
+    """Sender-visible time of one wave of fused epilogues (n_ctas CTAs each storing
+    bytes_per_cta, then a compute gap gap_ns before the next wave): the Burst-Gap prediction
+    max(T0_iss, V/R - G) and the completion-coupled one (the issuer waits V/R)."""
+    f = fit(points)
+    v = n_ctas * bytes_per_cta
+    t0 = t0_at(points, f["K_for_R"], v)
+    return {"V_bytes": v, "T0_ns": t0, "burst_gap_ns": predict(t0, f["R_GBps"], v, gap_ns),
+            "completion_coupled_ns": max(t0, completion_coupled(f["R_GBps"], v))}
+
+
+def fused_overhead_check(points, names=("mmdit", "long", "video"), reps: int = 15):
+    """Measured fused-minus-attention-only time against the two models, per workload."""
+    import torch
+
+    import ulysses_attention_output_b200 as xs
+    from ulysses_attention_output_b200 import workloads as W
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    out = []
+    for name in names:
+        w = W.WORKLOADS[name]
+        g = torch.Generator(device="cuda").manual_seed(0)
+        q, k, v = (torch.randn(w.shape(), generator=g, device="cuda").to(torch.bfloat16) for _ in range(3))
+        dest = xs.alloc_dest(w.B, w.H, w.S, w.D, w.P, device="cuda")
+        o = torch.empty_like(q)
+        # Alternate the two kernels call by call and take per-call medians, so that clock
+        # drift under the power cap affects both alike.
+        fns = {"fused": lambda: xs.attn_a2a_fused(q, k, v, dest), "attn_only": lambda: xs.attn(q, k, v, o)}
+        samples = {label: [] for label in fns}
+        for _ in range(3):
+            for fn in fns.values():
+                fn()
+        torch.cuda.synchronize()
+        for _ in range(reps):
+            for label, fn in fns.items():
+                e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+                e0.record()
+                fn()
+                e1.record()
+                torch.cuda.synchronize()
+                samples[label].append(e0.elapsed_time(e1) * 1e6)  # ns
+        times = {label: float(np.median(v)) for label, v in samples.items()}
+        n_items = w.B * w.H * ((w.S + 255) // 256)
+        waves = math.ceil(n_items / sms)
+        item_ns = times["attn_only"] / waves
+        m = epilogue_models(points, sms, 2 * 128 * w.D * 2, item_ns)
+        out.append({"workload": name, "S": w.S, "fused_ns": times["fused"],
+                    "attn_only_ns": times["attn_only"],
+                    "measured_overhead_ns": times["fused"] - times["attn_only"],
+                    "waves": waves, "item_ns": item_ns,
+                    "pred_burst_gap_exposed_ns": waves * max(0.0, m["burst_gap_ns"] - m["T0_ns"]),
+                    "pred_completion_coupled_exposed_ns": waves * m["completion_coupled_ns"],
+                    "model": m})
+        del q, k, v, dest, o
+    return out
+
+
+def main(argv=None):
+    argv = sys.argv[1:] if argv is None else argv
+    volumes = [4096 << i for i in range(11)]         # 4 KB .. 4 MB
+    producers = [1, 8, 32, 148]
+    gaps = [0] + [256 << i for i in range(9)]         # 0, 256 .. 65536 cycles
+    if "--large" in argv:                            # bursts beyond the default range
+        volumes = [4 << 20, 8 << 20, 16 << 20, 32 << 20, 64 << 20]
+        producers = [148]
+    threads = 1024 if "--wide" in argv else 256
+    pts = sweep(volumes, producers, gaps, threads=threads)
+    res = {"threads_per_producer": threads, "points": pts, "fit": fit(pts)}
+    if "--fused" in argv:
+        res["fused"] = fused_overhead_check(pts)
+    print(json.dumps(res))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
