@@ -204,7 +204,7 @@ class OracleSample:
     first few heads, each against all S keys of its head (the same seeded values the GPU arm
     uses)."""
 
-    def __init__(self, w, heads: int = 4):
+    def __init__(self, w, heads: int = 8, max_rows: int = 1024):
         import oracle
         from ulysses_attention_output_b200 import workloads as W
         self.oracle = oracle
@@ -213,7 +213,7 @@ class OracleSample:
         q, k, v = W.make_inputs(w)
         sl = (slice(0, 1), slice(0, self.heads))
         self.q, self.k, self.v = (t[sl].contiguous() for t in (q, k, v))
-        self.rows = W.sample_rows(w, n=min(w.S, 256)).numpy()[:1, :self.heads]
+        self.rows = W.sample_rows(w, n=min(w.S, max_rows)).numpy()[:1, :self.heads]
         self.threads = oracle.max_threads()
 
     def run(self, n: int) -> float:
