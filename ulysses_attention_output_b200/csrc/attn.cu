@@ -24,7 +24,8 @@
 // softmax overlaps the other tile's two MMAs.  The running maximum is only moved when a new
 // row maximum exceeds it by more than 2^8 (in the exp2 domain); P then stays below 256 and
 // the rescale of O (done by the softmax thread itself, after the previous P V completed) is
-// rare.  P V consumes the probabilities rounded to bf16, and l sums those same rounded values
+// rare (the previous P V is complete by then: it precedes the Q K^T whose result the
+// softmax has just read).  P V consumes the probabilities rounded to bf16, and l sums those same rounded values
 // in fp32, so the normalised weights of every row add up to one.  The softmax works on column
 // pairs in packed fp32 (f32x2) and computes 5 of every 16 pairs of exponentials with an FMA-pipe
 // polynomial instead of MUFU ex2, because at one exponential per 4*D FLOPs MUFU alone would
@@ -268,14 +269,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           ++pc0;
           ptx::tc_fence_after();
           issue_pv(0, slotV, j > 0);
-          ptx::mma_commit(o_done(0));
           const bool more = (j + 1) < n_kv;
+          // The s_full commit after QK_t(j+1) also covers PV_t(j), issued just before it, so
+          // o_done is only needed for the last key tile (the epilogue waits for it).
+          if (!more) ptx::mma_commit(o_done(0));
           if (more) {
             slotK = kv_it % kStages;
             ok = bounded_wait(kv_full(slotK), (kv_it / kStages) & 1u, ctl);
             if (!ok) break;
             ++kv_it;
-            ptx::tc_fence_after();
+            // (no tcgen05 fence here: K arrived through TMA, no tensor-memory hand-off)
             issue_qk(0, slotK);
             ptx::mma_commit(s_full(0));
             if (j + 2 == n_kv) ptx::mma_commit(q_empty(0));
@@ -285,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           ++pc1;
           ptx::tc_fence_after();
           issue_pv(1, slotV, j > 0);
-          ptx::mma_commit(o_done(1));
+          if (!more) ptx::mma_commit(o_done(1));
           ptx::mma_commit(kv_empty(slotV));
           if (more) {
             issue_qk(1, slotK);
@@ -313,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     uint8_t *stg = base + L::kStage + warp * (kStageRows * L::kStageRowBytes);
     uint8_t **rowptr = reinterpret_cast<uint8_t **>(base + L::kRowPtr) + warp * kStageRows;
     uint32_t sc = 0;       // s_full phases consumed
-    uint32_t pv_base = 0;  // P V products of this tile completed before the current item
+    uint32_t item_cnt = 0;  // work items finished by this CTA (o_done completes once per item)
     bool ok = true;
 
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
@@ -427,11 +430,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           l_run += (a0 + a1) + (b0 + b1);
         }
         if (__any_sync(0xffffffffu, rescale)) {
-          // O holds P V of the previous key tiles: wait for the last of them, then scale.
-          ok = bounded_wait(o_done(t), (pv_base + j - 1) & 1u, ctl);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          ptx::tc_fence_after();
+          // O holds P V of the previous key tiles, all complete: PV_t(j-1) was issued before
+          // QK_t(j), whose completion (s_full) this thread has waited for.
           const float a = rescale ? alpha : 1.f;
 #pragma unroll
           for (int cc = 0; cc < DCH * 2; ++cc) {
@@ -452,10 +452,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       if (!ok) break;
 
       // ---------------------------------------------------------- epilogue
-      ok = bounded_wait(o_done(t), (pv_base + n_kv - 1) & 1u, ctl);
+      ok = bounded_wait(o_done(t), item_cnt & 1u, ctl);  // the item's last P V
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      pv_base += n_kv;
+      ++item_cnt;
       ptx::tc_fence_after();
       const float inv_l = 1.f / l_run;
       // Destination of this thread's row.
