@@ -77,6 +77,26 @@ XS_API xs_status xs_attn_a2a_fused(const void *q, const void *k, const void *v, 
                             xs_shape shape, float scale, xs_stream_t stream, int *dev_status);
 
 /*
+ * The same fused call for one rank of a multi-GPU Ulysses layer (the per-rank piece of the
+ * exchange the pages describe: each rank owns a subset of the heads over the full sequence
+ * and writes its finished tiles into every rank's sequence shard).
+ *   q, k, v     : device, [B, shape.H, S, D]: the shape.H heads this rank owns.
+ *   heads_total : heads of the layer; every destination row holds all of them.
+ *   head_offset : global index of this rank's first head (rank g of P: g * shape.H).
+ *   dest        : HOST array of shape.P slab pointers; dest[r] is [B, S/P, heads_total, D].
+ *                 The pointers may be this GPU's memory or memory of other GPUs that this
+ *                 GPU can store to (peer access); the call only stores to them.
+ * Writes dest[r][b, s_local, head_offset + h, :] = O[b, h, r*S/P + s_local, :] for this
+ * rank's heads h; the other heads' columns of the slabs are left untouched.  Requires
+ * heads_total % P == 0, S % P == 0 and head_offset + shape.H <= heads_total.
+ * xs_attn_a2a_fused(...) equals this call with heads_total = shape.H, head_offset = 0.
+ */
+XS_API xs_status xs_attn_a2a_fused_rank(const void *q, const void *k, const void *v,
+                                        void *const *dest, xs_shape shape, int heads_total,
+                                        int head_offset, float scale, xs_stream_t stream,
+                                        int *dev_status);
+
+/*
  * Attention only, head-major output: out[b,h,s,:] (device, [B, H, S, D] bf16).  The same
  * kernel and arithmetic as xs_attn_a2a_fused, so out re-laid by xs_a2a_relayout equals the
  * fused result bit for bit.  First half of the serial baseline the pages compare against
@@ -93,6 +113,18 @@ XS_API xs_status xs_attn(const void *q, const void *k, const void *v, void *out,
  */
 XS_API xs_status xs_a2a_relayout(const void *src, void *const *dest, xs_shape shape,
                           xs_stream_t stream);
+
+/*
+ * The pre-attention All-to-All of Ulysses (sequence shards -> head-major; the direction
+ * that precedes the attention in the layer the pages fuse the post-attention exchange
+ * into):
+ *   dst[b, h, r*S/P + s_local, :] = src[r][b, s_local, head_offset + h, :]
+ * for h < heads_local (one rank's heads; heads_local = H and head_offset = 0 gathers all).
+ * src: host array of P device slab pointers, each [B, S/P, H, D] with H = shape.H (all heads);
+ * dst: device [B, heads_local, S, D].  A pure copy of 16-bit words.
+ */
+XS_API xs_status xs_a2a_pre(void *const *src, void *dst, xs_shape shape, int heads_local,
+                            int head_offset, xs_stream_t stream);
 
 /*
  * Burst-Gap store microbenchmark (explainer, "Methodik: Die X-Stage-Abstraktion und das

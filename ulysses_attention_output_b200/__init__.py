@@ -9,6 +9,8 @@ Calls (same names as the C ABI, without the ``xs_`` prefix):
 * :func:`attn_a2a_fused` -- attention fused with the post-attention exchange into P slabs.
 * :func:`attn`           -- attention with a head-major output.
 * :func:`a2a_relayout`   -- the exchange as a separate pass (serial baseline).
+* :func:`attn_a2a_fused_rank` -- the fused call of one Ulysses rank (its heads, all slabs).
+* :func:`a2a_pre`        -- the pre-attention exchange (sequence shards -> head-major).
 * :func:`burst_probe`    -- Burst-Gap store microbenchmark.
 * :func:`burst_probe_static` -- the same, with no device allocation (fixed library scratch).
 * :func:`selftest_bounded_wait` -- exercises the bounded on-device wait.
@@ -22,6 +24,7 @@ import threading
 __all__ = [
     "XsError", "XS_OK", "XS_ERR_INVALID_ARG", "XS_ERR_UNSUPPORTED", "XS_ERR_CUDA", "XS_ERR_TIMEOUT",
     "library_path", "load", "version", "attn_a2a_fused", "attn", "a2a_relayout", "burst_probe",
+    "attn_a2a_fused_rank", "a2a_pre",
     "burst_probe_static", "selftest_bounded_wait", "alloc_dest", "HostPipeline", "attention_flops",
 ]
 
@@ -76,12 +79,15 @@ def load():
         ip = ctypes.c_void_p  # device int*
         lib.xs_attn_a2a_fused.argtypes = [vp, vp, vp, vpp, Shape, c_float, vp, ip]
         lib.xs_attn.argtypes = [vp, vp, vp, vp, Shape, c_float, vp, ip]
+        lib.xs_attn_a2a_fused_rank.argtypes = [vp, vp, vp, vpp, Shape, c_int, c_int, c_float, vp, ip]
+        lib.xs_a2a_pre.argtypes = [vpp, vp, Shape, c_int, c_int, vp]
         lib.xs_a2a_relayout.argtypes = [vp, vpp, Shape, vp]
         lib.xs_burst_probe.argtypes = [vp, ctypes.c_longlong, BurstCfg, vp, vp]
         lib.xs_burst_probe_static.argtypes = [BurstCfg, vp, vp]
         lib.xs_selftest_bounded_wait.argtypes = [ip, ctypes.c_longlong, vp]
         for fn in (lib.xs_attn_a2a_fused, lib.xs_attn, lib.xs_a2a_relayout, lib.xs_burst_probe,
-                   lib.xs_burst_probe_static, lib.xs_selftest_bounded_wait):
+                   lib.xs_burst_probe_static, lib.xs_selftest_bounded_wait,
+                   lib.xs_attn_a2a_fused_rank, lib.xs_a2a_pre):
             fn.restype = c_int
         lib.xs_get_error_string.argtypes = [c_int]
         lib.xs_get_error_string.restype = ctypes.c_char_p
@@ -158,6 +164,36 @@ def attn_a2a_fused(q, k, v, dest, scale: float | None = None, stream=None, statu
     arr = _dest_array(dest, shp)
     _check(load().xs_attn_a2a_fused(q.data_ptr(), k.data_ptr(), v.data_ptr(), arr, shp,
                                     float(scale or 0.0), _stream_handle(stream), _ptr(status)))
+
+
+def attn_a2a_fused_rank(q, k, v, dest, heads_total: int, head_offset: int, scale: float | None = None,
+                        stream=None, status=None):
+    """One Ulysses rank's fused call: its heads ``q, k, v`` [B, H_rank, S, D] scattered into
+    every rank's slab ``dest[r]`` [B, S/P, heads_total, D] at heads head_offset .. +H_rank."""
+    P = len(dest)
+    shp = _shape_of(q, P)
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _bf16_cuda(n, t, tuple(q.shape))
+    for r, d in enumerate(dest):
+        _bf16_cuda(f"dest[{r}]", d, (shp.B, shp.S // P, int(heads_total), shp.D))
+    arr = (ctypes.c_void_p * P)(*[d.data_ptr() for d in dest])
+    _check(load().xs_attn_a2a_fused_rank(q.data_ptr(), k.data_ptr(), v.data_ptr(), arr, shp,
+                                         int(heads_total), int(head_offset), float(scale or 0.0),
+                                         _stream_handle(stream), _ptr(status)))
+
+
+def a2a_pre(src, dst, heads_local: int | None = None, head_offset: int = 0, stream=None):
+    """Pre-attention exchange: P sequence-shard slabs ``src[r]`` [B, S/P, H, D] -> head-major
+    ``dst`` [B, heads_local, S, D] holding heads head_offset .. head_offset + heads_local."""
+    P = len(src)
+    B, Sl, H, D = (int(x) for x in src[0].shape)
+    heads_local = H if heads_local is None else int(heads_local)
+    for r, t in enumerate(src):
+        _bf16_cuda(f"src[{r}]", t, (B, Sl, H, D))
+    _bf16_cuda("dst", dst, (B, heads_local, Sl * P, D))
+    arr = (ctypes.c_void_p * P)(*[t.data_ptr() for t in src])
+    _check(load().xs_a2a_pre(arr, dst.data_ptr(), Shape(B, H, Sl * P, D, P), heads_local,
+                             int(head_offset), _stream_handle(stream)))
 
 
 def attn(q, k, v, out, scale: float | None = None, stream=None, status=None, P: int = 1):

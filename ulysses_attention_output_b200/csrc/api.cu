@@ -96,9 +96,11 @@ xs_status check_inputs(const void *q, const void *k, const void *v, const xs_sha
   return XS_OK;
 }
 
-xs_status check_dest(void *const *dest, const xs_shape &s, const void *const *inputs, int n_inputs) {
+xs_status check_dest(void *const *dest, const xs_shape &s, const void *const *inputs, int n_inputs,
+                     int heads_total = -1) {
   if (!dest) return fail(XS_ERR_INVALID_ARG, "dest must be a host array of P device pointers");
-  const uintptr_t slab = static_cast<uintptr_t>(s.B) * (s.S / s.P) * s.H * s.D * 2;
+  const int hd = heads_total > 0 ? heads_total : s.H;
+  const uintptr_t slab = static_cast<uintptr_t>(s.B) * (s.S / s.P) * hd * s.D * 2;
   const uintptr_t full = static_cast<uintptr_t>(s.B) * s.H * s.S * s.D * 2;
   for (int r = 0; r < s.P; ++r) {
     if (!dest[r]) return fail(XS_ERR_INVALID_ARG, "dest[%d] is null", r);
@@ -127,6 +129,8 @@ xs_status fill_attention(xs::AttnParams &p, const void *q, const void *k, const 
   p.S = s.S;
   p.D = s.D;
   p.P = s.P;
+  p.H_dest = s.H;
+  p.head_offset = 0;
   p.S_local = s.S / s.P;
   p.n_kv = (s.S + 127) / 128;
   p.n_pairs = (s.S + 255) / 256;
@@ -175,6 +179,33 @@ xs_status xs_attn_a2a_fused(const void *q, const void *k, const void *v, void *c
                   "attention launch");
 }
 
+xs_status xs_attn_a2a_fused_rank(const void *q, const void *k, const void *v, void *const *dest,
+                                 xs_shape shape, int heads_total, int head_offset, float scale,
+                                 xs_stream_t stream, int *dev_status) {
+  // Per-rank form: shape.H heads of this rank; H % P is not required here (the layer's
+  // heads_total is), the destination rows hold heads_total heads.
+  xs_shape layer = shape;
+  layer.H = heads_total;
+  xs_status st = check_shape(layer, true);
+  if (st != XS_OK) return st;
+  if ((st = check_shape(shape, false)) != XS_OK) return st;
+  if (shape.S % shape.P != 0)
+    return fail(XS_ERR_UNSUPPORTED, "S %% P != 0 (S=%d P=%d)", shape.S, shape.P);
+  if (head_offset < 0 || shape.H > heads_total || head_offset > heads_total - shape.H)
+    return fail(XS_ERR_INVALID_ARG, "heads [%d, %d) are not inside the layer's %d heads", head_offset,
+                head_offset + shape.H, heads_total);
+  if ((st = check_inputs(q, k, v, shape)) != XS_OK) return st;
+  const void *ins[3] = {q, k, v};
+  if ((st = check_dest(dest, shape, ins, 3, heads_total)) != XS_OK) return st;
+  xs::AttnParams p;
+  if ((st = fill_attention(p, q, k, v, shape, scale, dev_status)) != XS_OK) return st;
+  p.H_dest = heads_total;
+  p.head_offset = head_offset;
+  for (int r = 0; r < shape.P; ++r) p.dest[r] = dest[r];
+  return launched(xs::launch_attention(p, xs::kSeqScatter, reinterpret_cast<cudaStream_t>(stream)),
+                  "attention launch");
+}
+
 xs_status xs_attn(const void *q, const void *k, const void *v, void *out, xs_shape shape,
                   float scale, xs_stream_t stream, int *dev_status) {
   xs_status st = check_shape(shape, false);
@@ -213,6 +244,38 @@ xs_status xs_a2a_relayout(const void *src, void *const *dest, xs_shape shape, xs
   p.P = shape.P;
   p.S_local = shape.S / shape.P;
   return launched(xs::launch_relayout(p, reinterpret_cast<cudaStream_t>(stream)), "relayout launch");
+}
+
+xs_status xs_a2a_pre(void *const *src, void *dst, xs_shape shape, int heads_local, int head_offset,
+                     xs_stream_t stream) {
+  xs_status st = check_shape(shape, true);
+  if (st != XS_OK) return st;
+  if (heads_local <= 0 || head_offset < 0 || head_offset > shape.H - heads_local)
+    return fail(XS_ERR_INVALID_ARG, "heads [%d, %d) are not inside the layer's %d heads", head_offset,
+                head_offset + heads_local, shape.H);
+  if (!dst || !aligned16(dst)) return fail(XS_ERR_INVALID_ARG, "dst must be a 16-byte aligned device pointer");
+  if (!src) return fail(XS_ERR_INVALID_ARG, "src must be a host array of P device pointers");
+  const uintptr_t slab = static_cast<uintptr_t>(shape.B) * (shape.S / shape.P) * shape.H * shape.D * 2;
+  const uintptr_t out_bytes = static_cast<uintptr_t>(shape.B) * heads_local * shape.S * shape.D * 2;
+  const Range o{reinterpret_cast<uintptr_t>(dst), reinterpret_cast<uintptr_t>(dst) + out_bytes};
+  xs::PreRelayoutParams p;
+  std::memset(&p, 0, sizeof(p));
+  for (int r = 0; r < shape.P; ++r) {
+    if (!src[r] || !aligned16(src[r])) return fail(XS_ERR_INVALID_ARG, "src[%d] is null or not 16-byte aligned", r);
+    const Range a{reinterpret_cast<uintptr_t>(src[r]), reinterpret_cast<uintptr_t>(src[r]) + slab};
+    if (overlap(a, o)) return fail(XS_ERR_INVALID_ARG, "src[%d] overlaps dst", r);
+    p.src[r] = src[r];
+  }
+  p.dst = dst;
+  p.B = shape.B;
+  p.H_total = shape.H;
+  p.H_local = heads_local;
+  p.head_offset = head_offset;
+  p.S = shape.S;
+  p.D = shape.D;
+  p.P = shape.P;
+  p.S_local = shape.S / shape.P;
+  return launched(xs::launch_pre_relayout(p, reinterpret_cast<cudaStream_t>(stream)), "pre-exchange launch");
 }
 
 xs_status xs_burst_probe(void *scratch, long long scratch_bytes, xs_burst_cfg cfg,

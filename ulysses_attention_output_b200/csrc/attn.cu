@@ -467,11 +467,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     (static_cast<size_t>(bh) * p.S + s_row) * static_cast<size_t>(D) * 2;
         } else {
           const int b = bh / p.H;
-          const int h = bh - b * p.H;
+          const int h = bh - b * p.H + p.head_offset;  // global head index
           const int r = s_row / p.S_local;
           const int sl = s_row - r * p.S_local;
           dst_row = static_cast<uint8_t *>(p.dest[r]) +
-                    ((static_cast<size_t>(b) * p.S_local + sl) * p.H + h) * static_cast<size_t>(D) * 2;
+                    ((static_cast<size_t>(b) * p.S_local + sl) * p.H_dest + h) * static_cast<size_t>(D) * 2;
         }
       }
       // Two rounds of 16 rows per warp: stage rows in shared memory (chunk order rotated by

@@ -50,6 +50,48 @@ __global__ void __launch_bounds__(256) relayout_kernel(const __grid_constant__ R
   }
 }
 
+// ---------------------------------------------------------------- pre-attention exchange
+// dst[b, h, r*S_local + s_local, :] = src[r][b, s_local, head_offset + h, :], h < H_local.
+// One warp per source row (r, b, s_local): H_local*D contiguous words of src[r], written as
+// H_local runs of D words into the head-major dst.  16-byte loads and stores, four in flight.
+__global__ void __launch_bounds__(256) pre_relayout_kernel(const __grid_constant__ PreRelayoutParams p) {
+  const int nch = p.D >> 3;
+  const int row_chunks = p.H_local * nch;
+  const long long rows_per_rank = static_cast<long long>(p.B) * p.S_local;
+  const long long n_rows = rows_per_rank * p.P;
+  const int lane = threadIdx.x & 31;
+  const long long warp0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  uint4 *dst = static_cast<uint4 *>(p.dst);
+  const long long head_stride = static_cast<long long>(p.S) * nch;  // chunks between heads of dst
+  for (long long row = warp0; row < n_rows; row += n_warps) {
+    const int r = static_cast<int>(row / rows_per_rank);
+    const long long rem = row - r * rows_per_rank;
+    const int b = static_cast<int>(rem / p.S_local);
+    const int sl = static_cast<int>(rem - static_cast<long long>(b) * p.S_local);
+    const int s = r * p.S_local + sl;
+    const uint4 *src = static_cast<const uint4 *>(p.src[r]) +
+                       (rem * p.H_total + p.head_offset) * nch;
+    uint4 *db = dst + (static_cast<long long>(b) * p.H_local * p.S + s) * nch;
+    int i = lane;
+    for (; i + 96 < row_chunks; i += 128) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = __ldg(src + i + 32 * u);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int ii = i + 32 * u;
+        const int h = ii / nch;
+        db[h * head_stride + (ii - h * nch)] = v[u];
+      }
+    }
+    for (; i < row_chunks; i += 32) {
+      const int h = i / nch;
+      db[h * head_stride + (i - h * nch)] = __ldg(src + i);
+    }
+  }
+}
+
 // ---------------------------------------------------------------- Burst-Gap probe
 // Each CTA is one producer.  Per burst: stamp, every thread issues its part of the
 // producer's share of 16-byte stores, the CTA syncs (all stores issued, none waited for),
@@ -145,6 +187,18 @@ cudaError_t launch_relayout(const RelayoutParams &p, cudaStream_t stream) {
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   relayout_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pre_relayout(const PreRelayoutParams &p, cudaStream_t stream) {
+  const int sms = device_sm_count();
+  if (sms <= 0) return cudaErrorInvalidDevice;
+  const long long n_rows = static_cast<long long>(p.B) * p.S_local * p.P;
+  long long blocks = (n_rows + 7) / 8;
+  const long long cap = static_cast<long long>(sms) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  pre_relayout_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -68,7 +68,9 @@ struct AttnParams {
   CUtensorMap tm_v;
   void *out;               // kHeadMajor
   void *dest[kMaxRanks];   // kSeqScatter
-  int B, H, S, D, P;
+  int B, H, S, D, P;       // H = heads held by this call (the rank's heads)
+  int H_dest;              // heads per destination row (all heads of the layer)
+  int head_offset;         // global index of this call's first head
   int S_local;             // S / P
   int n_kv;                // ceil(S / 128)
   int n_pairs;             // ceil(S / 256): work items per (b, h)
@@ -89,6 +91,13 @@ struct RelayoutParams {
   int B, H, S, D, P, S_local;
 };
 cudaError_t launch_relayout(const RelayoutParams &p, cudaStream_t stream);
+
+struct PreRelayoutParams {
+  const void *src[kMaxRanks];  // P sequence-shard slabs [B, S/P, H_total, D]
+  void *dst;                   // head-major [B, H_local, S, D]
+  int B, H_total, H_local, head_offset, S, D, P, S_local;
+};
+cudaError_t launch_pre_relayout(const PreRelayoutParams &p, cudaStream_t stream);
 
 struct BurstParams {
   uint4 *scratch;
