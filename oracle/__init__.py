@@ -19,6 +19,15 @@ Communication-Computation Overlap in DiT Inference"; abstract, and the explainer
 * :func:`dest_slot`   -- where one output row lands.
 * :func:`softmax_row` -- the normalised probabilities of one query row.
 
+Partial attention and its merge follow the page "Move the Query, Not the Cache:
+Characterizing Cross-Instance Latent Attention Redistribution Across GPU Fabrics" (explainer
+"Technisches Resuemee: Den Query bewegen, nicht den Cache" -> "Methodik" -> "Primitiv-Vergleich",
+the Route primitive, and "Korrektheitsverifizierung"):
+
+* :func:`attention_partial` -- attention of the query rows over one key/value shard, with the
+  row's log-sum-exp ``lse = log sum_j exp(s_j)``.
+* :func:`lse_merge`         -- the online-softmax merge of partial results of disjoint shards.
+
 All are pinned by ``tests/test_oracle_pins.py`` against closed forms, invariants, hand-made
 fixtures under ``tests/golden/`` and an independent numpy brute force.
 """
@@ -75,6 +84,11 @@ def _load():
                                                              ctypes.POINTER(ctypes.c_longlong)]
             lib.xs_oracle_dest_slot.restype = c_int
             lib.xs_oracle_max_threads.restype = c_int
+            lib.xs_oracle_attention_partial.argtypes = [dp, dp, dp, c_int, c_int, c_int, c_int, c_int,
+                                                        ctypes.c_double, ip, c_int, dp, dp, c_int]
+            lib.xs_oracle_attention_partial.restype = c_int
+            lib.xs_oracle_lse_merge.argtypes = [dp, dp, c_int, ctypes.c_longlong, c_int, dp, dp]
+            lib.xs_oracle_lse_merge.restype = c_int
             _lib = lib
     return _lib
 
@@ -181,3 +195,64 @@ def dest_slot(B: int, H: int, S: int, D: int, P: int, b: int, h: int, s: int) ->
     if rc != 0:
         raise ValueError("xs_oracle_dest_slot rejected its arguments")
     return int(r.value), int(off.value)
+
+
+def _rows_arg(rows, B: int, H: int):
+    rows_arr = np.asarray(rows, dtype=np.int32)
+    if rows_arr.ndim == 1:
+        rows_arr = np.broadcast_to(rows_arr, (B, H, rows_arr.shape[0]))
+    rows_arr = np.ascontiguousarray(rows_arr.reshape(B, H, -1), dtype=np.int32)
+    return rows_arr, rows_arr.shape[2], rows_arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+def attention_partial(q, k, v, scale: float | None = None, rows=None, nthreads: int = 0):
+    """fp64 partial attention of q [B,H,Sq,D] over one key/value shard k, v [B,H,Skv,D].
+
+    Returns ``(out [B,H,n,D], lse [B,H,n])`` with n = Sq or len(rows); lse is the natural-log
+    log-sum-exp of the scaled scores.  Skv may be 0 (then out = 0 and lse = -inf).
+    ``scale`` defaults to 1/sqrt(D).
+    """
+    lib = _load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    if q.ndim != 4 or k.ndim != 4 or v.shape != k.shape or k.shape[:2] != q.shape[:2] \
+            or k.shape[3] != q.shape[3]:
+        raise ValueError(f"need q [B,H,Sq,D] and k, v [B,H,Skv,D]; got {q.shape} {k.shape} {v.shape}")
+    B, H, Sq, D = q.shape
+    Skv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    if rows is None:
+        n, rows_arr, rows_ptr = Sq, None, ctypes.POINTER(ctypes.c_int32)()
+    else:
+        rows_arr, n, rows_ptr = _rows_arg(rows, B, H)
+    out = np.empty((B, H, n, D), dtype=np.float64)
+    lse = np.empty((B, H, n), dtype=np.float64)
+    kk = k if Skv > 0 else np.zeros(1)
+    vv = v if Skv > 0 else np.zeros(1)
+    rc = lib.xs_oracle_attention_partial(_dp(q), _dp(kk), _dp(vv), B, H, Sq, Skv, D, float(scale),
+                                         rows_ptr, n, _dp(out), _dp(lse), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"xs_oracle_attention_partial rejected its arguments (rc={rc})")
+    return out, lse
+
+
+def lse_merge(o_parts, lse_parts):
+    """fp64 online-softmax merge of n partial results.
+
+    o_parts: [n, ..., D]; lse_parts: [n, ...] (same leading shape; -inf marks an empty part).
+    Returns ``(out [..., D], lse [...])``.
+    """
+    lib = _load()
+    o = _f64(o_parts)
+    lse = _f64(lse_parts)
+    if o.ndim < 2 or lse.shape != o.shape[:-1]:
+        raise ValueError(f"need o_parts [n, ..., D] and lse_parts [n, ...]; got {o.shape} {lse.shape}")
+    n, D = o.shape[0], o.shape[-1]
+    lead = o.shape[1:-1]
+    R = int(np.prod(lead)) if lead else 1
+    out = np.empty(lead + (D,), dtype=np.float64)
+    lse_out = np.empty(lead, dtype=np.float64)
+    rc = lib.xs_oracle_lse_merge(_dp(o), _dp(lse), n, R, D, _dp(out), _dp(lse_out))
+    if rc != 0:
+        raise ValueError("xs_oracle_lse_merge rejected its arguments")
+    return out, lse_out

@@ -218,3 +218,140 @@ int xs_oracle_dest_slot(int B, int H, int S, int D, int P, int b, int h, int s, 
   *offset = (((long long)b * Sl + (s % Sl)) * H + h) * (long long)D;
   return XSO_OK;
 }
+
+/*
+ * 4. Partial attention over one key/value shard, returning the log-sum-exp of the row
+ *    (the "Route" primitive: the owner of a KV shard attends the routed query rows over its
+ *    own keys and sends back a small result that the requester merges with an online
+ *    softmax).  Source: page "Move the Query, Not the Cache: Characterizing Cross-Instance
+ *    Latent Attention Redistribution Across GPU Fabrics", explainer "Technisches Resuemee:
+ *    Den Query bewegen, nicht den Cache" -> "Methodik" -> "Primitiv-Vergleich" (Route) and
+ *    "Korrektheitsverifizierung" (routed partial attention merged by online softmax
+ *    reproduces single-instance attention).  The pages print no formula; the definitions
+ *    below are the textbook ones.  Per (b, h) and query row i, over the Skv keys j of the
+ *    shard:
+ *         s_j = scale * sum_d q[b,h,i,d] * k[b,h,j,d]
+ *         m   = max_j s_j
+ *         l   = sum_j exp(s_j - m)
+ *         O_i = sum_j exp(s_j - m) * v[b,h,j,d] / l
+ *         lse = m + log(l)            (= log sum_j exp(s_j), natural log)
+ *    A shard without keys (Skv = 0) has l = 0: lse = -inf, and O is set to 0 (reading: the
+ *    empty part has weight zero in the merge, so its O never matters).
+ *
+ * 5. Merge of n partial results of the same query row (definition 4 applied to disjoint key
+ *    sets K_1 .. K_n whose union is all keys):
+ *         M   = max_t lse_t
+ *         w_t = exp(lse_t - M)
+ *         O   = sum_t w_t * O_t / sum_t w_t
+ *         lse = M + log(sum_t w_t)
+ *    which equals definition 1 (and 4) over the union, since w_t * O_t * exp(M) is the
+ *    un-normalised sum over K_t.  Rows whose parts are all empty (M = -inf) give O = 0 and
+ *    lse = -inf.
+ */
+
+/* One query row of definition 4.  k, v: [Skv, D]; work: [Skv] scratch. */
+static void partial_row(const double *q_row, const double *k, const double *v, int Skv, int D,
+                        double scale, double *out_row, double *lse, double *work) {
+  if (Skv == 0) {
+    for (int d = 0; d < D; ++d) out_row[d] = 0.0;
+    *lse = -INFINITY;
+    return;
+  }
+  double m = -INFINITY;
+  for (int j = 0; j < Skv; ++j) {
+    double dot = 0.0;
+    for (int d = 0; d < D; ++d) dot += q_row[d] * k[(size_t)j * D + d];
+    work[j] = dot * scale;
+    if (work[j] > m) m = work[j];
+  }
+  double l = 0.0;
+  for (int j = 0; j < Skv; ++j) {
+    work[j] = exp(work[j] - m);
+    l += work[j];
+  }
+  for (int d = 0; d < D; ++d) {
+    double acc = 0.0;
+    for (int j = 0; j < Skv; ++j) acc += work[j] * v[(size_t)j * D + d];
+    out_row[d] = acc / l;
+  }
+  *lse = m + log(l);
+}
+
+/*
+ * Partial attention (definition 4) for selected query rows of every (b, h).
+ *   q      : [B, H, Sq, D] fp64;  k, v: [B, H, Skv, D] fp64 (Skv may be 0: k, v unused).
+ *   rows   : NULL -> every row 0..Sq-1 (nrows must equal Sq); else [B*H, nrows] indices.
+ *   out    : [B, H, nrows, D];  lse: [B, H, nrows].
+ */
+int xs_oracle_attention_partial(const double *q, const double *k, const double *v, int B, int H,
+                                int Sq, int Skv, int D, double scale, const int32_t *rows,
+                                int nrows, double *out, double *lse, int nthreads) {
+  if (!q || !out || !lse || B <= 0 || H <= 0 || Sq <= 0 || Skv < 0 || D <= 0 || nrows <= 0)
+    return XSO_BAD_ARG;
+  if (Skv > 0 && (!k || !v)) return XSO_BAD_ARG;
+  if (!rows && nrows != Sq) return XSO_BAD_ARG;
+  if (rows) {
+    for (long long t = 0; t < (long long)B * H * nrows; ++t)
+      if (rows[t] < 0 || rows[t] >= Sq) return XSO_BAD_ARG;
+  }
+  const long long total = (long long)B * H * nrows;
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+  (void)nthreads;
+#endif
+  int fail = 0;
+#pragma omp parallel
+  {
+    double *work = (double *)malloc(sizeof(double) * (size_t)(Skv > 0 ? Skv : 1));
+    if (!work) {
+#pragma omp atomic write
+      fail = 1;
+    } else {
+#pragma omp for schedule(dynamic, 16)
+      for (long long t = 0; t < total; ++t) {
+        long long bh = t / nrows;
+        int ii = (int)(t % nrows);
+        int i = rows ? rows[bh * nrows + ii] : ii;
+        const double *kb = Skv > 0 ? k + (size_t)bh * Skv * D : NULL;
+        const double *vb = Skv > 0 ? v + (size_t)bh * Skv * D : NULL;
+        partial_row(q + ((size_t)bh * Sq + i) * D, kb, vb, Skv, D, scale, out + (size_t)t * D,
+                    lse + t, work);
+      }
+      free(work);
+    }
+  }
+  return fail ? XSO_BAD_ARG : XSO_OK;
+}
+
+/*
+ * Merge (definition 5) of n partial results.
+ *   o_parts  : [n, R, D] fp64;  lse_parts: [n, R] fp64 (-inf marks an empty part).
+ *   out      : [R, D];  lse_out: [R] (nullable).
+ */
+int xs_oracle_lse_merge(const double *o_parts, const double *lse_parts, int n, long long R, int D,
+                        double *out, double *lse_out) {
+  if (!o_parts || !lse_parts || !out || n <= 0 || R <= 0 || D <= 0) return XSO_BAD_ARG;
+  for (long long r = 0; r < R; ++r) {
+    double M = -INFINITY;
+    for (int t = 0; t < n; ++t)
+      if (lse_parts[(size_t)t * R + r] > M) M = lse_parts[(size_t)t * R + r];
+    double *o = out + (size_t)r * D;
+    if (M == -INFINITY) {
+      for (int d = 0; d < D; ++d) o[d] = 0.0;
+      if (lse_out) lse_out[r] = -INFINITY;
+      continue;
+    }
+    double W = 0.0;
+    for (int d = 0; d < D; ++d) o[d] = 0.0;
+    for (int t = 0; t < n; ++t) {
+      const double w = exp(lse_parts[(size_t)t * R + r] - M);
+      W += w;
+      const double *ot = o_parts + ((size_t)t * R + r) * D;
+      for (int d = 0; d < D; ++d) o[d] += w * ot[d];
+    }
+    for (int d = 0; d < D; ++d) o[d] /= W;
+    if (lse_out) lse_out[r] = M + log(W);
+  }
+  return XSO_OK;
+}
