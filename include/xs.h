@@ -127,6 +127,47 @@ XS_API xs_status xs_a2a_pre(void *const *src, void *dst, xs_shape shape, int hea
                             int head_offset, xs_stream_t stream);
 
 /*
+ * Partial attention over one key/value shard, with the log-sum-exp of every query row: the
+ * owner's side of the Route primitive (page "Move the Query, Not the Cache: Characterizing
+ * Cross-Instance Latent Attention Redistribution Across GPU Fabrics", explainer "Technisches
+ * Resuemee: Den Query bewegen, nicht den Cache" -> "Methodik" -> "Primitiv-Vergleich": the
+ * query is sent to the owner of a KV shard, the owner computes the partial attention there,
+ * and the requester merges the small results by online softmax).  Per (b, h) and query row i,
+ * over the s_kv keys j of the shard, with s_j = scale * q[b,h,i,:] . k[b,h,j,:]:
+ *   o_part[b,h,i,:] = sum_j exp(s_j) v[b,h,j,:] / sum_j exp(s_j)
+ *   lse[b,h,i]      = log sum_j exp(s_j)                         (natural log)
+ *   q      : device [B, H, S, D] bf16 (S = shape.S query rows);
+ *   k, v   : device [B, H, s_kv, D] bf16 (unused, may be NULL, when s_kv == 0);
+ *   o_part : device [B, H, S, D] fp32, 16-byte aligned;  lse: device [B, H, S] fp32.
+ * shape.P must be 1 (no exchange here); the other shape rules are those of xs_attn, with any
+ * s_kv >= 0 (ragged tails masked).  s_kv == 0 (an empty shard) writes o_part = 0 and
+ * lse = -inf, which the merge treats as a part of weight zero.  Numerics: as xs_attn (P
+ * rounded to bf16 before P V, fp32 accumulation, l summed from the rounded weights), the
+ * output kept in fp32 so that the merge adds no bf16 rounding of its own.
+ */
+XS_API xs_status xs_attn_partial(const void *q, const void *k, const void *v, float *o_part,
+                                 float *lse, xs_shape shape, int s_kv, float scale,
+                                 xs_stream_t stream, int *dev_status);
+
+/*
+ * The requester's merge of n_parts partial results of the same query rows over disjoint key
+ * shards (same passage as xs_attn_partial): per row, M = max_t lse_t, w_t = exp(lse_t - M),
+ *   out = sum_t w_t o_t / sum_t w_t            (rounded to bf16)
+ *   lse_out = M + log(sum_t w_t)               (when lse_out is not NULL)
+ * which is the attention over the union of the shards.  Rows whose parts all have
+ * lse = -inf give out = 0 and lse_out = -inf; a part with lse = -inf has no weight.
+ *   o_parts   : host array of n_parts device pointers, each [rows, D] fp32, 16-byte aligned;
+ *   lse_parts : host array of n_parts device pointers, each [rows] fp32;
+ *   out       : device [rows, D] bf16;  lse_out: device [rows] fp32 or NULL.
+ * 1 <= n_parts <= XS_MAX_PARTS; D % 8 == 0, 8 <= D <= 4096.  Outputs may not overlap inputs.
+ * For partial attention results, rows = B * H * S (their [B, H, S] leading dimensions).
+ */
+#define XS_MAX_PARTS 16
+XS_API xs_status xs_lse_merge(const float *const *o_parts, const float *const *lse_parts,
+                              int n_parts, void *out, float *lse_out, long long rows, int D,
+                              xs_stream_t stream);
+
+/*
  * Burst-Gap store microbenchmark (explainer, "Methodik: Die X-Stage-Abstraktion und das
  * Burst-Gap-Modell": sender-visible issue time T_iss(G; K, V) of a burst of volume V from K
  * producers separated by a compute gap G).  Each of `producers` CTAs repeats n_bursts times:

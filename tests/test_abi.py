@@ -116,3 +116,27 @@ def test_product_never_imports_oracle():
                 text = open(os.path.join(dirpath, fn)).read()
                 assert "import oracle" not in text and "from oracle" not in text, fn
                 assert "xs_oracle" not in text, fn
+
+
+def test_partial_and_merge_reject(lib):
+    sh = xs.Shape(1, 4, 256, 64, 1)
+    q, k, v, o, l = FAKE, FAKE + MB, FAKE + 2 * MB, FAKE + 8 * MB, FAKE + 16 * MB
+    P = lib.xs_attn_partial
+    assert P(q, k, v, o, l, xs.Shape(1, 4, 256, 64, 2), 128, 0.0, None, None) == xs.XS_ERR_INVALID_ARG  # P != 1
+    assert P(q, k, v, o, l, sh, -1, 0.0, None, None) == xs.XS_ERR_INVALID_ARG            # negative s_kv
+    assert P(q, k, v, o, l, xs.Shape(1, 4, 256, 136, 1), 128, 0.0, None, None) == xs.XS_ERR_UNSUPPORTED
+    assert P(q, 0, v, o, l, sh, 128, 0.0, None, None) == xs.XS_ERR_INVALID_ARG            # k missing
+    assert P(q, k, v, o + 4, l, sh, 128, 0.0, None, None) == xs.XS_ERR_INVALID_ARG        # o misaligned
+    assert P(q, k, v, o, o + 1024, sh, 128, 0.0, None, None) == xs.XS_ERR_INVALID_ARG     # lse inside o
+    assert P(q, k, v, q + 1024, l, sh, 128, 0.0, None, None) == xs.XS_ERR_INVALID_ARG     # o overlaps q
+    M = lib.xs_lse_merge
+    op = (ctypes.c_void_p * 2)(FAKE, FAKE + 4 * MB)
+    lp = (ctypes.c_void_p * 2)(FAKE + 8 * MB, FAKE + 9 * MB)
+    out = FAKE + 16 * MB
+    assert M(op, lp, 0, out, None, 1024, 128, None) == xs.XS_ERR_UNSUPPORTED              # no parts
+    assert M(op, lp, 17, out, None, 1024, 128, None) == xs.XS_ERR_UNSUPPORTED             # too many
+    assert M(op, lp, 2, out, None, 1024, 100, None) == xs.XS_ERR_UNSUPPORTED              # D % 8
+    assert M(op, lp, 2, out, None, 0, 128, None) == xs.XS_ERR_INVALID_ARG                 # no rows
+    assert M(op, lp, 2, FAKE + 1024, None, 1024, 128, None) == xs.XS_ERR_INVALID_ARG      # out inside part 0
+    bad = (ctypes.c_void_p * 2)(FAKE + 4, FAKE + 4 * MB)
+    assert M(bad, lp, 2, out, None, 1024, 128, None) == xs.XS_ERR_INVALID_ARG             # misaligned part

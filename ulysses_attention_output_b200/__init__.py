@@ -11,6 +11,8 @@ Calls (same names as the C ABI, without the ``xs_`` prefix):
 * :func:`a2a_relayout`   -- the exchange as a separate pass (serial baseline).
 * :func:`attn_a2a_fused_rank` -- the fused call of one Ulysses rank (its heads, all slabs).
 * :func:`a2a_pre`        -- the pre-attention exchange (sequence shards -> head-major).
+* :func:`attn_partial`   -- partial attention over one key/value shard, fp32 output + lse.
+* :func:`lse_merge`      -- online-softmax merge of partial results (the Route primitive).
 * :func:`burst_probe`    -- Burst-Gap store microbenchmark.
 * :func:`burst_probe_static` -- the same, with no device allocation (fixed library scratch).
 * :func:`selftest_bounded_wait` -- exercises the bounded on-device wait.
@@ -24,7 +26,7 @@ import threading
 __all__ = [
     "XsError", "XS_OK", "XS_ERR_INVALID_ARG", "XS_ERR_UNSUPPORTED", "XS_ERR_CUDA", "XS_ERR_TIMEOUT",
     "library_path", "load", "version", "attn_a2a_fused", "attn", "a2a_relayout", "burst_probe",
-    "attn_a2a_fused_rank", "a2a_pre",
+    "attn_a2a_fused_rank", "a2a_pre", "attn_partial", "lse_merge",
     "burst_probe_static", "selftest_bounded_wait", "alloc_dest", "HostPipeline", "attention_flops",
 ]
 
@@ -85,9 +87,11 @@ def load():
         lib.xs_burst_probe.argtypes = [vp, ctypes.c_longlong, BurstCfg, vp, vp]
         lib.xs_burst_probe_static.argtypes = [BurstCfg, vp, vp]
         lib.xs_selftest_bounded_wait.argtypes = [ip, ctypes.c_longlong, vp]
+        lib.xs_attn_partial.argtypes = [vp, vp, vp, vp, vp, Shape, c_int, c_float, vp, ip]
+        lib.xs_lse_merge.argtypes = [vpp, vpp, c_int, vp, vp, ctypes.c_longlong, c_int, vp]
         for fn in (lib.xs_attn_a2a_fused, lib.xs_attn, lib.xs_a2a_relayout, lib.xs_burst_probe,
                    lib.xs_burst_probe_static, lib.xs_selftest_bounded_wait,
-                   lib.xs_attn_a2a_fused_rank, lib.xs_a2a_pre):
+                   lib.xs_attn_a2a_fused_rank, lib.xs_a2a_pre, lib.xs_attn_partial, lib.xs_lse_merge):
             fn.restype = c_int
         lib.xs_get_error_string.argtypes = [c_int]
         lib.xs_get_error_string.restype = ctypes.c_char_p
@@ -203,6 +207,76 @@ def attn(q, k, v, out, scale: float | None = None, stream=None, status=None, P: 
         _bf16_cuda(n, t, tuple(q.shape))
     _check(load().xs_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), shp,
                           float(scale or 0.0), _stream_handle(stream), _ptr(status)))
+
+
+def _f32_cuda(name: str, t, shape):
+    import torch
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.float32:
+        raise TypeError(f"{name} must be a float32 torch.Tensor")
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def attn_partial(q, k, v, o_part=None, lse=None, scale: float | None = None, stream=None, status=None):
+    """Partial attention of ``q`` [B, H, S, D] over the key/value shard ``k, v`` [B, H, Skv, D].
+
+    Returns ``(o_part, lse)``: fp32 [B, H, S, D] (normalised over the shard's keys) and fp32
+    [B, H, S] (natural-log log-sum-exp of the scaled scores).  Outputs are allocated by
+    PyTorch when not given.  Skv may be 0.
+    """
+    import torch
+    shp = _shape_of(q, 1)
+    _bf16_cuda("q", q)
+    if k.dim() != 4 or tuple(k.shape[:2]) != (shp.B, shp.H) or int(k.shape[3]) != shp.D:
+        raise ValueError(f"k must be [B, H, Skv, D] matching q; got {tuple(k.shape)}")
+    s_kv = int(k.shape[2])
+    if s_kv > 0:
+        _bf16_cuda("k", k)
+        _bf16_cuda("v", v, tuple(k.shape))
+    if o_part is None:
+        o_part = torch.empty(tuple(q.shape), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty(tuple(q.shape[:3]), dtype=torch.float32, device=q.device)
+    _f32_cuda("o_part", o_part, tuple(q.shape))
+    _f32_cuda("lse", lse, tuple(q.shape[:3]))
+    kp = k.data_ptr() if s_kv > 0 else None
+    vp_ = v.data_ptr() if s_kv > 0 else None
+    _check(load().xs_attn_partial(q.data_ptr(), kp, vp_, o_part.data_ptr(), lse.data_ptr(), shp, s_kv,
+                                  float(scale or 0.0), _stream_handle(stream), _ptr(status)))
+    return o_part, lse
+
+
+def lse_merge(o_parts, lse_parts, out=None, lse_out=None, stream=None):
+    """Merge partial results: ``o_parts[t]`` fp32 [..., D], ``lse_parts[t]`` fp32 [...].
+
+    Returns ``out`` (bf16 [..., D]) and ``lse_out`` (fp32 [...]; pass ``lse_out=False`` to skip it).
+    """
+    import torch
+    n = len(o_parts)
+    if n != len(lse_parts) or n < 1:
+        raise ValueError("need as many lse parts as output parts, at least one")
+    lead = tuple(o_parts[0].shape[:-1])
+    D = int(o_parts[0].shape[-1])
+    for t in range(n):
+        _f32_cuda(f"o_parts[{t}]", o_parts[t], lead + (D,))
+        _f32_cuda(f"lse_parts[{t}]", lse_parts[t], lead)
+    if out is None:
+        out = torch.empty(lead + (D,), dtype=torch.bfloat16, device=o_parts[0].device)
+    _bf16_cuda("out", out, lead + (D,))
+    if lse_out is None:
+        lse_out = torch.empty(lead, dtype=torch.float32, device=o_parts[0].device)
+    if lse_out is not False:
+        _f32_cuda("lse_out", lse_out, lead)
+    rows = 1
+    for x in lead:
+        rows *= int(x)
+    op = (ctypes.c_void_p * n)(*[t.data_ptr() for t in o_parts])
+    lp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in lse_parts])
+    _check(load().xs_lse_merge(op, lp, n, out.data_ptr(), None if lse_out is False else lse_out.data_ptr(),
+                               rows, D, _stream_handle(stream)))
+    return out, (None if lse_out is False else lse_out)
 
 
 def a2a_relayout(src, dest, stream=None):

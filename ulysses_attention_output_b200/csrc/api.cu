@@ -54,13 +54,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // 3-D view {D, S, B*H} of a [B, H, S, D] bf16 tensor; box {64, 128, 1}; 128-byte swizzle;
 // out-of-range elements (D padding, rows past S) read as zero.
-bool make_qkv_map(CUtensorMap *m, const void *ptr, const xs_shape &s) {
+// `rows` is the S extent of the view (the key count for k and v of a partial attention).
+bool make_qkv_map(CUtensorMap *m, const void *ptr, const xs_shape &s, int rows) {
   auto enc = encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(s.D), static_cast<cuuint64_t>(s.S),
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(s.D), static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(s.B) * static_cast<cuuint64_t>(s.H)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(s.D) * 2,
-                           static_cast<cuuint64_t>(s.S) * static_cast<cuuint64_t>(s.D) * 2};
+                           static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(s.D) * 2};
   cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides,
@@ -118,10 +119,13 @@ xs_status check_dest(void *const *dest, const xs_shape &s, const void *const *in
   return XS_OK;
 }
 
+// s_kv: key/value rows (-1: the same as the query rows s.S).
 xs_status fill_attention(xs::AttnParams &p, const void *q, const void *k, const void *v,
-                         const xs_shape &s, float scale, int *dev_status) {
+                         const xs_shape &s, float scale, int *dev_status, int s_kv = -1) {
   std::memset(&p, 0, sizeof(p));
-  if (!make_qkv_map(&p.tm_q, q, s) || !make_qkv_map(&p.tm_k, k, s) || !make_qkv_map(&p.tm_v, v, s))
+  if (s_kv < 0) s_kv = s.S;
+  if (!make_qkv_map(&p.tm_q, q, s, s.S) || !make_qkv_map(&p.tm_k, k, s, s_kv) ||
+      !make_qkv_map(&p.tm_v, v, s, s_kv))
     return fail(XS_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point %s)",
                 encode_fn() ? "found" : "missing");
   p.B = s.B;
@@ -131,8 +135,9 @@ xs_status fill_attention(xs::AttnParams &p, const void *q, const void *k, const 
   p.P = s.P;
   p.H_dest = s.H;
   p.head_offset = 0;
+  p.S_kv = s_kv;
   p.S_local = s.S / s.P;
-  p.n_kv = (s.S + 127) / 128;
+  p.n_kv = (s_kv + 127) / 128;
   p.n_pairs = (s.S + 255) / 256;
   p.n_items = s.B * s.H * p.n_pairs;
   const double sc = scale > 0.f ? static_cast<double>(scale) : 1.0 / std::sqrt(static_cast<double>(s.D));
@@ -225,6 +230,84 @@ xs_status xs_attn(const void *q, const void *k, const void *v, void *out, xs_sha
   p.out = out;
   return launched(xs::launch_attention(p, xs::kHeadMajor, reinterpret_cast<cudaStream_t>(stream)),
                   "attention launch");
+}
+
+xs_status xs_attn_partial(const void *q, const void *k, const void *v, float *o_part, float *lse,
+                          xs_shape shape, int s_kv, float scale, xs_stream_t stream, int *dev_status) {
+  if (shape.P != 1) return fail(XS_ERR_INVALID_ARG, "partial attention takes shape.P == 1 (got %d)", shape.P);
+  xs_status st = check_shape(shape, false);
+  if (st != XS_OK) return st;
+  if (s_kv < 0) return fail(XS_ERR_INVALID_ARG, "negative key count s_kv=%d", s_kv);
+  if (static_cast<long long>(shape.B) * shape.H * s_kv * shape.D > (1LL << 40))
+    return fail(XS_ERR_UNSUPPORTED, "key/value shard of %d rows out of range", s_kv);
+  if (!q || !aligned16(q)) return fail(XS_ERR_INVALID_ARG, "q must be a 16-byte aligned device pointer");
+  if (s_kv > 0 && (!k || !v || !aligned16(k) || !aligned16(v)))
+    return fail(XS_ERR_INVALID_ARG, "k and v must be 16-byte aligned device pointers");
+  if (!o_part || !aligned16(o_part)) return fail(XS_ERR_INVALID_ARG, "o_part must be a 16-byte aligned device pointer");
+  if (!lse || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return fail(XS_ERR_INVALID_ARG, "lse must be a 4-byte aligned device pointer");
+  const uintptr_t rows = static_cast<uintptr_t>(shape.B) * shape.H * shape.S;
+  const Range ro{reinterpret_cast<uintptr_t>(o_part), reinterpret_cast<uintptr_t>(o_part) + rows * shape.D * 4};
+  const Range rl{reinterpret_cast<uintptr_t>(lse), reinterpret_cast<uintptr_t>(lse) + rows * 4};
+  if (overlap(ro, rl)) return fail(XS_ERR_INVALID_ARG, "o_part overlaps lse");
+  {
+    const Range rq{reinterpret_cast<uintptr_t>(q), reinterpret_cast<uintptr_t>(q) + rows * shape.D * 2};
+    const uintptr_t kv_bytes = static_cast<uintptr_t>(shape.B) * shape.H * s_kv * shape.D * 2;
+    for (const Range &o : {ro, rl}) {
+      if (overlap(o, rq)) return fail(XS_ERR_INVALID_ARG, "an output overlaps q");
+      for (const void *in : {k, v}) {
+        if (s_kv == 0) break;
+        const Range r{reinterpret_cast<uintptr_t>(in), reinterpret_cast<uintptr_t>(in) + kv_bytes};
+        if (overlap(o, r)) return fail(XS_ERR_INVALID_ARG, "an output overlaps k or v");
+      }
+    }
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (s_kv == 0)
+    return launched(xs::launch_partial_empty(o_part, lse, static_cast<long long>(rows), shape.D, s),
+                    "empty-shard fill launch");
+  xs::AttnParams p;
+  if ((st = fill_attention(p, q, k, v, shape, scale, dev_status, s_kv)) != XS_OK) return st;
+  p.out = o_part;
+  p.lse = lse;
+  return launched(xs::launch_attention(p, xs::kPartial, s), "partial attention launch");
+}
+
+xs_status xs_lse_merge(const float *const *o_parts, const float *const *lse_parts, int n_parts,
+                       void *out, float *lse_out, long long rows, int D, xs_stream_t stream) {
+  if (n_parts < 1 || n_parts > XS_MAX_PARTS)
+    return fail(XS_ERR_UNSUPPORTED, "n_parts=%d outside [1, %d]", n_parts, XS_MAX_PARTS);
+  if (rows < 1 || rows > (1LL << 36)) return fail(XS_ERR_INVALID_ARG, "rows=%lld out of range", rows);
+  if (D < 8 || D % 8 != 0 || D > 4096)
+    return fail(XS_ERR_UNSUPPORTED, "D=%d unsupported (need D %% 8 == 0, 8 <= D <= 4096)", D);
+  if (!o_parts || !lse_parts) return fail(XS_ERR_INVALID_ARG, "o_parts and lse_parts must be host arrays");
+  if (!out || !aligned16(out)) return fail(XS_ERR_INVALID_ARG, "out must be a 16-byte aligned device pointer");
+  if (lse_out && (reinterpret_cast<uintptr_t>(lse_out) & 3u))
+    return fail(XS_ERR_INVALID_ARG, "lse_out must be 4-byte aligned");
+  const Range ro{reinterpret_cast<uintptr_t>(out), reinterpret_cast<uintptr_t>(out) + rows * D * 2};
+  const Range rlo{reinterpret_cast<uintptr_t>(lse_out),
+                  reinterpret_cast<uintptr_t>(lse_out) + (lse_out ? rows * 4 : 0)};
+  if (lse_out && overlap(ro, rlo)) return fail(XS_ERR_INVALID_ARG, "out overlaps lse_out");
+  xs::MergeParams p;
+  std::memset(&p, 0, sizeof(p));
+  for (int t = 0; t < n_parts; ++t) {
+    if (!o_parts[t] || !aligned16(o_parts[t]))
+      return fail(XS_ERR_INVALID_ARG, "o_parts[%d] must be a 16-byte aligned device pointer", t);
+    if (!lse_parts[t] || (reinterpret_cast<uintptr_t>(lse_parts[t]) & 3u))
+      return fail(XS_ERR_INVALID_ARG, "lse_parts[%d] must be a 4-byte aligned device pointer", t);
+    const Range a{reinterpret_cast<uintptr_t>(o_parts[t]), reinterpret_cast<uintptr_t>(o_parts[t]) + rows * D * 4};
+    const Range b{reinterpret_cast<uintptr_t>(lse_parts[t]), reinterpret_cast<uintptr_t>(lse_parts[t]) + rows * 4};
+    if (overlap(a, ro) || overlap(b, ro) || (lse_out && (overlap(a, rlo) || overlap(b, rlo))))
+      return fail(XS_ERR_INVALID_ARG, "part %d overlaps an output", t);
+    p.o[t] = o_parts[t];
+    p.lse[t] = lse_parts[t];
+  }
+  p.n = n_parts;
+  p.out = out;
+  p.lse_out = lse_out;
+  p.rows = rows;
+  p.D = D;
+  return launched(xs::launch_lse_merge(p, reinterpret_cast<cudaStream_t>(stream)), "merge launch");
 }
 
 xs_status xs_a2a_relayout(const void *src, void *const *dest, xs_shape shape, xs_stream_t stream) {
@@ -322,6 +405,7 @@ xs_status xs_burst_probe_static(xs_burst_cfg cfg, unsigned long long *stamps, xs
                 "use xs_burst_probe with a caller-allocated buffer",
                 cfg.burst_bytes, static_cast<long long>(XS_BURST_STATIC_SCRATCH_BYTES));
   static_assert(XS_BURST_STATIC_SCRATCH_BYTES == xs::kStaticProbeScratchBytes, "scratch size mismatch");
+  static_assert(XS_MAX_PARTS == xs::kMaxParts, "part count mismatch");
   uint4 *scratch = nullptr;
   cudaError_t e = xs::static_probe_scratch(&scratch);
   if (e != cudaSuccess) return fail(XS_ERR_CUDA, "scratch address lookup: %s", cudaGetErrorString(e));

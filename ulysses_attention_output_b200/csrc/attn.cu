@@ -10,6 +10,12 @@
 // which is the gap in which the issued stores drain.  No warp or SM is dedicated to the
 // exchange: the same warps that ran the softmax write the tile and go on.
 //
+// A third epilogue writes the partial attention of the query rows over one key/value shard
+// (S_kv keys) in fp32 together with each row's log-sum-exp, for the Route primitive of the
+// page "Move the Query, Not the Cache: Characterizing Cross-Instance Latent Attention
+// Redistribution Across GPU Fabrics" ("Methodik" -> "Primitiv-Vergleich"): the owner of a
+// KV shard attends the routed queries over its keys and the requester merges the results.
+//
 // Structure of one persistent CTA (320 threads, one CTA per SM):
 //   warps 0-3  softmax for Q tile 0 (one thread per query row = one TMEM lane)
 //   warps 4-7  softmax for Q tile 1
@@ -331,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         if (!ok) break;
         ++sc;
         ptx::tc_fence_after();
-        const int kv_valid = p.S - j * 128;  // < 128 only on a ragged last key tile
+        const int kv_valid = p.S_kv - j * 128;  // < 128 only on a ragged last key tile
         // Pass 1: row maximum over the 128 scores (one TMEM round trip for the whole row).
         float m0, m1, m2, m3;
         {
@@ -462,30 +468,41 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       const int s_row = q0 + 128 * t + row;
       uint8_t *dst_row = nullptr;
       if (s_row < p.S) {
-        if constexpr (EPI == kHeadMajor) {
-          dst_row = static_cast<uint8_t *>(p.out) +
-                    (static_cast<size_t>(bh) * p.S + s_row) * static_cast<size_t>(D) * 2;
-        } else {
+        if constexpr (EPI == kSeqScatter) {
           const int b = bh / p.H;
           const int h = bh - b * p.H + p.head_offset;  // global head index
           const int r = s_row / p.S_local;
           const int sl = s_row - r * p.S_local;
           dst_row = static_cast<uint8_t *>(p.dest[r]) +
                     ((static_cast<size_t>(b) * p.S_local + sl) * p.H_dest + h) * static_cast<size_t>(D) * 2;
+        } else {
+          constexpr size_t kOutBytes = EPI == kPartial ? 4 : 2;
+          dst_row = static_cast<uint8_t *>(p.out) +
+                    (static_cast<size_t>(bh) * p.S + s_row) * static_cast<size_t>(D) * kOutBytes;
+        }
+        if constexpr (EPI == kPartial) {
+          // log sum_j exp(scale * s_j) = ln 2 * (m + log2 l), m and l in the exp2 domain
+          // (l sums the same bf16-rounded weights that P V used).
+          p.lse[static_cast<size_t>(bh) * p.S + s_row] = (m_run + log2f(l_run)) * 0.69314718055994531f;
         }
       }
-      // Two rounds of 16 rows per warp: stage rows in shared memory (chunk order rotated by
-      // row to spread banks), then write whole rows with consecutive lanes on consecutive
-      // 16-byte chunks.  The stores are not waited for: the warp goes straight on to its
-      // next tile while they drain.
+      // Rounds of kRows rows per warp (16 in bf16, 8 in fp32): stage rows in shared memory
+      // (chunk order rotated by row to spread banks), then write whole rows with consecutive
+      // lanes on consecutive 16-byte chunks.  The stores are not waited for: the warp goes
+      // straight on to its next tile while they drain.
       // O is read from TMEM once per round, 32 columns at a time (the warp-collective load
       // brings all 32 rows; the lanes of the current round keep theirs).
+      constexpr int kEB = EPI == kPartial ? 4 : 2;        // bytes per output element
+      constexpr int kRows = kStageRows * 2 / kEB;          // rows per round
+      constexpr int kRowBytes = L::kStageRowBytes * kEB / 2;
+      constexpr int kChunksPerLd = 2 * kEB;                // 16-byte chunks per 32 columns
+      const int nch = D * kEB / 16;                        // 16-byte chunks per output row
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const bool mine = (lane >> 4) == half;
-        const int r16 = lane & 15;
-        const int rot = r16 % nch;
-        uint8_t *my = stg + r16 * L::kStageRowBytes;
+      for (int rd = 0; rd < 32 / kRows; ++rd) {
+        const bool mine = lane / kRows == rd;
+        const int rr = lane % kRows;
+        const int rot = rr % nch;
+        uint8_t *my = stg + rr * kRowBytes;
 #pragma unroll
         for (int cc = 0; cc < DCH * 2; ++cc) {
           uint32_t o[32];
@@ -494,30 +511,34 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           ptx::reg_fence32(o);
           if (mine) {
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              const int c = cc * 4 + q4;  // 16-byte chunk (8 columns) of the output row
+            for (int q4 = 0; q4 < kChunksPerLd; ++q4) {
+              const int c = cc * kChunksPerLd + q4;  // 16-byte chunk of the output row
               if (c < nch) {
                 int pc = c + rot;
                 if (pc >= nch) pc -= nch;
                 uint32_t w[4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                  w[i] = ptx::pack_bf16(u2f(o[8 * q4 + 2 * i]) * inv_l, u2f(o[8 * q4 + 2 * i + 1]) * inv_l);
+                for (int i = 0; i < 4; ++i) {
+                  if constexpr (kEB == 2)
+                    w[i] = ptx::pack_bf16(u2f(o[8 * q4 + 2 * i]) * inv_l, u2f(o[8 * q4 + 2 * i + 1]) * inv_l);
+                  else
+                    w[i] = f2u(u2f(o[4 * q4 + i]) * inv_l);
+                }
                 *reinterpret_cast<uint4 *>(my + pc * 16) = make_uint4(w[0], w[1], w[2], w[3]);
               }
             }
           }
         }
-        if (mine) rowptr[r16] = dst_row;
+        if (mine) rowptr[rr] = dst_row;
         __syncwarp();
-        for (int idx = lane; idx < kStageRows * nch; idx += 32) {
-          const int r16 = idx / nch;
-          const int c = idx - r16 * nch;
-          uint8_t *dr = rowptr[r16];
+        for (int idx = lane; idx < kRows * nch; idx += 32) {
+          const int r2 = idx / nch;
+          const int c = idx - r2 * nch;
+          uint8_t *dr = rowptr[r2];
           if (dr != nullptr) {
-            int pc = c + r16 % nch;
+            int pc = c + r2 % nch;
             if (pc >= nch) pc -= nch;
-            const uint4 v = *reinterpret_cast<const uint4 *>(stg + r16 * L::kStageRowBytes + pc * 16);
+            const uint4 v = *reinterpret_cast<const uint4 *>(stg + r2 * kRowBytes + pc * 16);
             ptx::st_global_v4(dr + c * 16, v);
           }
         }
@@ -564,9 +585,11 @@ size_t attention_smem_bytes(int dch) { return dch == 1 ? Smem<1>::kAlloc : Smem<
 cudaError_t launch_attention(const AttnParams &p, int epilogue, cudaStream_t stream) {
   const int dch = p.D <= 64 ? 1 : 2;
   if (dch == 1)
-    return epilogue == kHeadMajor ? launch_impl<1, kHeadMajor>(p, stream)
+    return epilogue == kHeadMajor  ? launch_impl<1, kHeadMajor>(p, stream)
+           : epilogue == kPartial ? launch_impl<1, kPartial>(p, stream)
                                   : launch_impl<1, kSeqScatter>(p, stream);
-  return epilogue == kHeadMajor ? launch_impl<2, kHeadMajor>(p, stream)
+  return epilogue == kHeadMajor  ? launch_impl<2, kHeadMajor>(p, stream)
+         : epilogue == kPartial ? launch_impl<2, kPartial>(p, stream)
                                 : launch_impl<2, kSeqScatter>(p, stream);
 }
 

@@ -60,19 +60,22 @@ __device__ __forceinline__ bool bounded_wait_drain(uint32_t bar, uint32_t parity
 enum EpilogueKind : int {
   kHeadMajor = 0,   // out[b, h, s, :]
   kSeqScatter = 1,  // dest[r][b, s_local, h, :]  (fused post-attention All-to-All)
+  kPartial = 2,     // out[b, h, s, :] in fp32 plus lse[b, h, s] (partial attention of a shard)
 };
 
 struct AttnParams {
   CUtensorMap tm_q;  // 3-D view {D, S, B*H} of q, box {64, 128, 1}, 128-byte swizzle
   CUtensorMap tm_k;
   CUtensorMap tm_v;
-  void *out;               // kHeadMajor
+  void *out;               // kHeadMajor (bf16), kPartial (fp32)
+  float *lse;              // kPartial: natural-log log-sum-exp of each query row
   void *dest[kMaxRanks];   // kSeqScatter
-  int B, H, S, D, P;       // H = heads held by this call (the rank's heads)
+  int B, H, S, D, P;       // H = heads held by this call (the rank's heads); S = query rows
+  int S_kv;                // key/value rows (= S except for partial attention over a shard)
   int H_dest;              // heads per destination row (all heads of the layer)
   int head_offset;         // global index of this call's first head
   int S_local;             // S / P
-  int n_kv;                // ceil(S / 128)
+  int n_kv;                // ceil(S_kv / 128), >= 1
   int n_pairs;             // ceil(S / 256): work items per (b, h)
   int n_items;             // B * H * n_pairs
   float scale_log2;        // softmax scale * log2(e)
@@ -116,6 +119,21 @@ constexpr long long kStaticProbeScratchBytes = 32LL << 20;
 cudaError_t static_probe_scratch(uint4 **out);
 
 cudaError_t launch_wait_selftest(int *status, long long limit_ns, cudaStream_t stream);
+
+// ---------------------------------------------------------------- log-sum-exp merge
+constexpr int kMaxParts = 16;
+struct MergeParams {
+  const float *o[kMaxParts];    // n partial outputs [rows, D] fp32
+  const float *lse[kMaxParts];  // n log-sum-exps [rows] fp32 (-inf = empty part)
+  int n;
+  void *out;                    // [rows, D] bf16
+  float *lse_out;               // [rows] fp32, nullable
+  long long rows;
+  int D;
+};
+cudaError_t launch_lse_merge(const MergeParams &p, cudaStream_t stream);
+// Result of partial attention over zero keys: o = 0, lse = -inf for `rows` rows of D.
+cudaError_t launch_partial_empty(float *o, float *lse, long long rows, int D, cudaStream_t stream);
 
 int device_sm_count();
 

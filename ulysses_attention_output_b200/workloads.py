@@ -137,3 +137,70 @@ def sample_rows(w: Workload, n: int | None = None, seed: int | None = None) -> t
                     seen.add(i)
             out[b, h] = torch.tensor(sorted(chosen), dtype=torch.int32)
     return out
+
+
+# ----------------------------------------------------------------------------- Route workloads
+@dataclass(frozen=True)
+class RouteWorkload:
+    """Partial attention of routed query rows over KV shards held by several owners, merged by
+    online softmax (the Route primitive).  ``shards`` lists each owner's key count."""
+    name: str
+    B: int
+    H: int
+    Sq: int
+    shards: tuple
+    D: int
+    seed: int = 0
+    sampled_rows: int = 0           # 0: every query row is checked against the oracle
+    description: str = field(default="", compare=False)
+
+    @property
+    def S_kv(self) -> int:
+        return int(sum(self.shards))
+
+    @property
+    def flops(self) -> int:
+        """Algorithmic FLOPs of the partial attentions: 4 * B * H * Sq * S_kv * D."""
+        return 4 * self.B * self.H * self.Sq * self.S_kv * self.D
+
+    @property
+    def merge_bytes(self) -> int:
+        """Algorithmic bytes of the merge: every part's fp32 O and lse read, bf16 O and fp32
+        lse written."""
+        rows = self.B * self.H * self.Sq
+        return len(self.shards) * rows * (4 * self.D + 4) + rows * (2 * self.D + 4)
+
+
+ROUTE_WORKLOADS: dict[str, RouteWorkload] = {
+    "route_tiny": RouteWorkload("route_tiny", 1, 2, 300, (256, 0, 411, 333), 128, 1005, 0,
+                                "Route check: 300 query rows, 4 owners (one empty), ragged shards"),
+    "route": RouteWorkload("route", 1, 32, 1024, (8192, 8192, 8192, 8192), 128, 1006, 64,
+                           "Route batched dispatch: B=1 H=32, 1024 query rows per head, "
+                           "4 owners x 8192 keys, D=128"),
+}
+
+
+def make_route_inputs(w: RouteWorkload):
+    """(q, [k_t], [v_t]) as contiguous bf16 CPU tensors: q [B, H, Sq, D], then per shard t
+    k_t and v_t [B, H, shards[t], D], all drawn fp32 N(0, 1) in that order and rounded."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(w.seed))
+    q = torch.randn((w.B, w.H, w.Sq, w.D), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    ks, vs = [], []
+    for n in w.shards:
+        ks.append(torch.randn((w.B, w.H, n, w.D), generator=g, dtype=torch.float32).to(torch.bfloat16))
+        vs.append(torch.randn((w.B, w.H, n, w.D), generator=g, dtype=torch.float32).to(torch.bfloat16))
+    return q.contiguous(), ks, vs
+
+
+def sample_route_rows(w: RouteWorkload, n: int | None = None, seed: int = 4321) -> torch.Tensor:
+    """Query rows to check per (b, h): int32 [B, H, n], sorted, always with rows 0 and Sq-1."""
+    n = max(2, w.sampled_rows if n is None else n)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    out = torch.empty((w.B, w.H, n), dtype=torch.int32)
+    for b in range(w.B):
+        for h in range(w.H):
+            rest = [i for i in torch.randperm(w.Sq, generator=g).tolist() if i not in (0, w.Sq - 1)]
+            out[b, h] = torch.tensor(sorted([0, w.Sq - 1] + rest[:n - 2]), dtype=torch.int32)
+    return out
