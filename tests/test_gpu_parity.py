@@ -64,6 +64,8 @@ SMALL_SHAPES = [
     (1, 2, 640, 16, 2, "iid"),      # D=16
     (1, 2, 300, 48, 2, "iid"),      # D=48
     (1, 3, 1000, 120, 1, "iid"),    # D=120, P=1
+    (1, 2, 256, 80, 2, "iid"),      # D=80: five of eight K steps carry data
+    (1, 2, 384, 112, 2, "iid"),     # D=112: seven of eight K steps carry data
 ]
 
 

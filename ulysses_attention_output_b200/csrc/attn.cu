@@ -211,8 +211,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const int ks_qk = (p.D + 15) >> 4;             // K steps of 16 for Q K^T (true D)
-      const uint32_t n_pv = static_cast<uint32_t>(ks_qk * 16);  // N of P V (D padded to 16)
+      const int ks_d = (p.D + 15) >> 4;              // K steps of 16 covering the true D
+      const uint32_t n_pv = static_cast<uint32_t>(ks_d * 16);   // N of P V (D padded to 16)
       const uint32_t idesc_qk = ptx::idesc_bf16_f32(128, 128, 0);
       const uint32_t idesc_pv = ptx::idesc_bf16_f32(128, n_pv, 1);
       uint32_t kv_it = 0, it = 0, pc0 = 0, pc1 = 0;
@@ -226,6 +226,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       const uint64_t dv0 = ptx::smem_desc_sw128(sKV, kChunkBytes, 1024);
       constexpr uint64_t kTileDesc = L::kTile >> 4;  // one tile, in descriptor address units
 
+      // Every K step of the padded D (DCH * 64) is issued, also when D is smaller: TMA fills
+      // Q and K beyond D with zeros, so those steps add exact zeros to S.  No MMA is issued
+      // under a run-time condition (instances of this kernel that did so computed a wrong S
+      // for D = 72 .. 112 in some builds).
       auto issue_qk = [&](int t, uint32_t slot) {
         const uint64_t a = dq0 + static_cast<uint64_t>(t) * kTileDesc;
         const uint64_t b = dk0 + static_cast<uint64_t>(slot) * kTileDesc;
@@ -233,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 #pragma unroll
         for (int ks = 0; ks < DCH * 4; ++ks) {
           const uint64_t off = static_cast<uint64_t>(((ks >> 2) * kChunkBytes + (ks & 3) * 32) >> 4);
-          if (ks < ks_qk) ptx::mma_ss(d, a + off, b + off, idesc_qk, ks > 0 ? 1u : 0u);
+          ptx::mma_ss(d, a + off, b + off, idesc_qk, ks > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, uint32_t slot, bool acc) {
