@@ -97,6 +97,24 @@ XS_API xs_status xs_attn_a2a_fused_rank(const void *q, const void *k, const void
                                         int *dev_status);
 
 /*
+ * xs_attn_a2a_fused with a record of the sender-visible store-issue span of every output
+ * tile (the quantity the X-Stage explainer's Burst-Gap model describes: "Methodik: Die
+ * X-Stage-Abstraktion und das Burst-Gap-Modell").  Same arguments and results as
+ * xs_attn_a2a_fused, plus:
+ *   spans     : device, 8-byte aligned, [n_items][2][4][3] uint64 with n_items = B * H *
+ *               ceil(S / 256) work items of 256 query rows (two 128-row tiles), for each
+ *               tile and each of the four warps that store it: SM clock (clock64) before the
+ *               warp prepares its first store, SM clock after its last 16-byte store has
+ *               been issued (not completed), and the global timer (ns) at the first stamp.
+ *   spans_len : words available at spans (>= n_items * 24, else XS_ERR_INVALID_ARG).
+ * A separate kernel instance: xs_attn_a2a_fused itself records nothing.
+ */
+XS_API xs_status xs_attn_a2a_fused_spans(const void *q, const void *k, const void *v,
+                                         void *const *dest, xs_shape shape, float scale,
+                                         unsigned long long *spans, long long spans_len,
+                                         xs_stream_t stream, int *dev_status);
+
+/*
  * Attention only, head-major output: out[b,h,s,:] (device, [B, H, S, D] bf16).  The same
  * kernel and arithmetic as xs_attn_a2a_fused, so out re-laid by xs_a2a_relayout equals the
  * fused result bit for bit.  First half of the serial baseline the pages compare against

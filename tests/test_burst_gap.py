@@ -68,3 +68,28 @@ def test_epilogue_models():
     # no gap: the drain term wins
     z = bg.epilogue_models(pts, 148, 65536, gap_ns=0.0)["burst_gap_ns"]
     assert abs(z - max(m["T0_ns"], v / 700.0)) < 1e-9 * z
+
+
+def test_span_stats_from_synthetic_stamps():
+    # 2 CTAs, 3 items each (items striped: i on CTA i % 2); SM clock 2 GHz.
+    ghz, grid, n = 2.0, 2, 6
+    st = np.zeros((n, 2, 4, 3), dtype=np.int64)
+    item_cycles = 100_000
+    for i in range(n):
+        c, k = i % grid, i // grid
+        for t in range(2):
+            for w in range(4):
+                t0 = 1_000 + k * item_cycles + 50 * w + 5_000 * t   # warps start staggered
+                st[i, t, w, 0] = t0
+                st[i, t, w, 1] = t0 + 2_000 + 100 * w               # last warp ends latest
+                st[i, t, w, 2] = int(t0 / ghz) + 10_000_000 * c
+    r = bg.span_stats(st, grid)
+    assert abs(r["ghz"] - ghz) < 1e-3
+    # span = max end - min start = (150 + 2000 + 300) - 0 = 2450 cycles = 1225 ns for every tile
+    assert r["tiles"] == 12
+    assert abs(r["span_ns"]["p50"] - 1225.0) < 1e-6 and abs(r["span_ns"]["p99"] - 1225.0) < 1e-6
+    # gap: next item's first start - this item's last end = 100000 - 2450 cycles
+    assert abs(r["gap_ns_median"] - (item_cycles - 2450) / ghz) < 1e-6
+    assert sum(r["hist_counts"]) == 12
+    # an explicit clock rate overrides the estimate
+    assert abs(bg.span_stats(st, grid, ghz=1.0)["span_ns"]["p50"] - 2450.0) < 1e-6

@@ -10,6 +10,7 @@ Calls (same names as the C ABI, without the ``xs_`` prefix):
 * :func:`attn`           -- attention with a head-major output.
 * :func:`a2a_relayout`   -- the exchange as a separate pass (serial baseline).
 * :func:`attn_a2a_fused_rank` -- the fused call of one Ulysses rank (its heads, all slabs).
+* :func:`attn_a2a_fused_spans` -- the fused call, also recording each tile's store-issue span.
 * :func:`a2a_pre`        -- the pre-attention exchange (sequence shards -> head-major).
 * :func:`attn_partial`   -- partial attention over one key/value shard, fp32 output + lse.
 * :func:`lse_merge`      -- online-softmax merge of partial results (the Route primitive).
@@ -26,7 +27,7 @@ import threading
 __all__ = [
     "XsError", "XS_OK", "XS_ERR_INVALID_ARG", "XS_ERR_UNSUPPORTED", "XS_ERR_CUDA", "XS_ERR_TIMEOUT",
     "library_path", "load", "version", "attn_a2a_fused", "attn", "a2a_relayout", "burst_probe",
-    "attn_a2a_fused_rank", "a2a_pre", "attn_partial", "lse_merge",
+    "attn_a2a_fused_rank", "a2a_pre", "attn_partial", "lse_merge", "attn_a2a_fused_spans",
     "burst_probe_static", "selftest_bounded_wait", "alloc_dest", "HostPipeline", "attention_flops",
 ]
 
@@ -88,10 +89,12 @@ def load():
         lib.xs_burst_probe_static.argtypes = [BurstCfg, vp, vp]
         lib.xs_selftest_bounded_wait.argtypes = [ip, ctypes.c_longlong, vp]
         lib.xs_attn_partial.argtypes = [vp, vp, vp, vp, vp, Shape, c_int, c_float, vp, ip]
+        lib.xs_attn_a2a_fused_spans.argtypes = [vp, vp, vp, vpp, Shape, c_float, vp, ctypes.c_longlong, vp, ip]
         lib.xs_lse_merge.argtypes = [vpp, vpp, c_int, vp, vp, ctypes.c_longlong, c_int, vp]
         for fn in (lib.xs_attn_a2a_fused, lib.xs_attn, lib.xs_a2a_relayout, lib.xs_burst_probe,
                    lib.xs_burst_probe_static, lib.xs_selftest_bounded_wait,
-                   lib.xs_attn_a2a_fused_rank, lib.xs_a2a_pre, lib.xs_attn_partial, lib.xs_lse_merge):
+                   lib.xs_attn_a2a_fused_rank, lib.xs_a2a_pre, lib.xs_attn_partial, lib.xs_lse_merge,
+                   lib.xs_attn_a2a_fused_spans):
             fn.restype = c_int
         lib.xs_get_error_string.argtypes = [c_int]
         lib.xs_get_error_string.restype = ctypes.c_char_p
@@ -168,6 +171,27 @@ def attn_a2a_fused(q, k, v, dest, scale: float | None = None, stream=None, statu
     arr = _dest_array(dest, shp)
     _check(load().xs_attn_a2a_fused(q.data_ptr(), k.data_ptr(), v.data_ptr(), arr, shp,
                                     float(scale or 0.0), _stream_handle(stream), _ptr(status)))
+
+
+def attn_a2a_fused_spans(q, k, v, dest, spans=None, scale: float | None = None, stream=None, status=None):
+    """``attn_a2a_fused`` that also records, for every work item (256 query rows), tile and
+    storing warp, the SM clock before its first store, the SM clock after its last store
+    was issued, and the global timer (ns): returns ``spans`` int64 [n_items, 2, 4, 3]."""
+    import torch
+    P = len(dest)
+    shp = _shape_of(q, P)
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _bf16_cuda(n, t, tuple(q.shape))
+    arr = _dest_array(dest, shp)
+    n_items = shp.B * shp.H * ((shp.S + 255) // 256)
+    if spans is None:
+        spans = torch.zeros((n_items, 2, 4, 3), dtype=torch.int64, device=q.device)
+    if spans.dtype != torch.int64 or not spans.is_cuda or not spans.is_contiguous():
+        raise ValueError("spans must be a contiguous int64 CUDA tensor")
+    _check(load().xs_attn_a2a_fused_spans(q.data_ptr(), k.data_ptr(), v.data_ptr(), arr, shp,
+                                          float(scale or 0.0), spans.data_ptr(), spans.numel(),
+                                          _stream_handle(stream), _ptr(status)))
+    return spans
 
 
 def attn_a2a_fused_rank(q, k, v, dest, heads_total: int, head_offset: int, scale: float | None = None,

@@ -25,11 +25,13 @@ ring in this GPU's memory, i.e. the local stand-in for remote stores) over a gri
 ``predict`` evaluates the model; ``completion_coupled`` is the counter-model in which the
 issuer waits until its stores have drained (issue time V / R for every burst, no overlap).
 
-Run ``python -m ulysses_attention_output_b200.burst_gap [--large] [--wide] [--fused]`` on a GPU
-for a sweep (``--large``: bursts of 4..64 MB from 148 producers; ``--wide``: 1024 threads per
-producer; ``--fused``: also time the fused kernel against attention alone on the MMDiT, long
-and video workloads and set the measured overhead beside both models' predictions); it
-prints one JSON object with the raw points and the fit.
+Run ``python -m ulysses_attention_output_b200.burst_gap [--large] [--wide] [--fused] [--spans]``
+on a GPU for a sweep (``--large``: bursts of 4..64 MB from 148 producers; ``--wide``: 1024
+threads per producer; ``--fused``: also time the fused kernel against attention alone on the
+MMDiT, long and video workloads and set the measured overhead beside both models'
+predictions; ``--spans``: the per-tile store-issue span histogram of the fused kernel,
+recorded by ``xs_attn_a2a_fused_spans``, beside both models' predictions); it prints one JSON
+object with the raw points and the fit.
 """
 from __future__ import annotations
 
@@ -203,6 +205,78 @@ def fused_overhead_check(points, names=("mmdit", "long", "video"), reps: int = 1
     return out
 
 
+def span_stats(spans, grid: int, ghz: float | None = None, bins: int = 30):
+    """Per-tile store-issue spans from the stamps of ``xs_attn_a2a_fused_spans``.
+
+    spans: [n_items, 2, 4, 3] (SM clock before the first store, SM clock after the last
+    store issue, global timer ns), items striped over ``grid`` CTAs (item i on CTA i % grid).
+    A tile's span runs from the earliest of its four warps' first stamps to the latest of
+    their second stamps (one SM clock).  The SM clock rate is taken from the stamps of CTAs
+    that ran several items (clock and timer deltas between their first and last item) unless
+    ``ghz`` is given.  The gap is the time from a tile's last store issue to the first store
+    of the next item's same tile on the same CTA (the compute gap G between its bursts).
+    """
+    st = np.asarray(spans, dtype=np.int64)
+    n = st.shape[0]
+    start = st[:, :, :, 0].min(axis=2)
+    end = st[:, :, :, 1].max(axis=2)
+    cyc = (end - start).astype(np.float64)            # [n_items, 2]
+    if ghz is None:
+        rates = []
+        for c in range(min(grid, n)):
+            items = np.arange(c, n, grid)
+            if len(items) < 2:
+                continue
+            d_clk = st[items[-1], 0, 0, 0] - st[items[0], 0, 0, 0]
+            d_ns = st[items[-1], 0, 0, 2] - st[items[0], 0, 0, 2]
+            if d_ns > 0 and d_clk > 0:
+                rates.append(d_clk / d_ns)
+        ghz = float(np.median(rates)) if rates else float("nan")
+    ns = cyc / ghz
+    gaps = []
+    for c in range(min(grid, n)):
+        items = np.arange(c, n, grid)
+        if len(items) >= 2:
+            gaps.append((start[items[1:], :] - end[items[:-1], :]).ravel())
+    gap_ns = np.concatenate(gaps) / ghz if gaps else np.array([])
+    flat = ns.ravel()
+    hist, edges = np.histogram(flat, bins=bins)
+    pct = {f"p{q}": float(np.percentile(flat, q)) for q in (10, 50, 90, 99)}
+    return {"ghz": ghz, "tiles": int(flat.size), "span_ns": pct, "span_mean_ns": float(flat.mean()),
+            "gap_ns_median": float(np.median(gap_ns)) if gap_ns.size else None,
+            "hist_counts": hist.tolist(), "hist_edges_ns": edges.tolist()}
+
+
+def store_spans(points, names=("mmdit", "long", "video")):
+    """Measured per-tile store-issue spans of the fused kernel against the Burst-Gap and the
+    completion-coupled predictions for one wave of tiles (every CTA storing one 128-row tile,
+    gap G = the measured median gap between a CTA's bursts)."""
+    import torch
+
+    import ulysses_attention_output_b200 as xs
+    from ulysses_attention_output_b200 import workloads as W
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    out = []
+    for name in names:
+        w = W.WORKLOADS[name]
+        g = torch.Generator(device="cuda").manual_seed(0)
+        q, k, v = (torch.randn(w.shape(), generator=g, device="cuda").to(torch.bfloat16) for _ in range(3))
+        dest = xs.alloc_dest(w.B, w.H, w.S, w.D, w.P, device="cuda")
+        xs.attn_a2a_fused(q, k, v, dest)
+        spans = xs.attn_a2a_fused_spans(q, k, v, dest)
+        torch.cuda.synchronize()
+        n_items = spans.shape[0]
+        stats = span_stats(spans.cpu().numpy(), min(n_items, sms))
+        tile_bytes = 128 * w.D * 2
+        gap = stats["gap_ns_median"] if stats["gap_ns_median"] is not None else 0.0
+        m = epilogue_models(points, min(n_items, sms), tile_bytes, gap)
+        out.append({"workload": name, "S": w.S, "tile_bytes": tile_bytes, "stats": stats,
+                    "pred_burst_gap_ns": m["burst_gap_ns"], "pred_completion_coupled_ns": m["completion_coupled_ns"],
+                    "pred_T0_ns": m["T0_ns"], "wave_bytes": m["V_bytes"]})
+        del q, k, v, dest, spans
+    return out
+
+
 def main(argv=None):
     argv = sys.argv[1:] if argv is None else argv
     volumes = [4096 << i for i in range(11)]         # 4 KB .. 4 MB
@@ -216,6 +290,8 @@ def main(argv=None):
     res = {"threads_per_producer": threads, "points": pts, "fit": fit(pts)}
     if "--fused" in argv:
         res["fused"] = fused_overhead_check(pts)
+    if "--spans" in argv:
+        res["spans"] = store_spans(pts)
     print(json.dumps(res))
     return 0
 

@@ -184,6 +184,41 @@ xs_status xs_attn_a2a_fused(const void *q, const void *k, const void *v, void *c
                   "attention launch");
 }
 
+xs_status xs_attn_a2a_fused_spans(const void *q, const void *k, const void *v, void *const *dest,
+                                  xs_shape shape, float scale, unsigned long long *spans,
+                                  long long spans_len, xs_stream_t stream, int *dev_status) {
+  xs_status st = check_shape(shape, true);
+  if (st != XS_OK) return st;
+  if ((st = check_inputs(q, k, v, shape)) != XS_OK) return st;
+  const void *ins[3] = {q, k, v};
+  if ((st = check_dest(dest, shape, ins, 3)) != XS_OK) return st;
+  xs::AttnParams p;
+  if ((st = fill_attention(p, q, k, v, shape, scale, dev_status)) != XS_OK) return st;
+  const long long need = static_cast<long long>(p.n_items) * 2 * 4 * 3;
+  if (!spans || (reinterpret_cast<uintptr_t>(spans) & 7u))
+    return fail(XS_ERR_INVALID_ARG, "spans must be an 8-byte aligned device pointer");
+  if (spans_len < need)
+    return fail(XS_ERR_INVALID_ARG, "spans holds %lld words, the call needs %lld (work items x 2 x 4 x 3)",
+                spans_len, need);
+  {
+    const Range rs{reinterpret_cast<uintptr_t>(spans), reinterpret_cast<uintptr_t>(spans) + need * 8};
+    const uintptr_t full = static_cast<uintptr_t>(shape.B) * shape.H * shape.S * shape.D * 2;
+    const uintptr_t slab = full / shape.P;
+    for (const void *in : {q, k, v}) {
+      const Range r{reinterpret_cast<uintptr_t>(in), reinterpret_cast<uintptr_t>(in) + full};
+      if (overlap(rs, r)) return fail(XS_ERR_INVALID_ARG, "spans overlaps an input tensor");
+    }
+    for (int r = 0; r < shape.P; ++r) {
+      const Range d{reinterpret_cast<uintptr_t>(dest[r]), reinterpret_cast<uintptr_t>(dest[r]) + slab};
+      if (overlap(rs, d)) return fail(XS_ERR_INVALID_ARG, "spans overlaps dest[%d]", r);
+    }
+  }
+  for (int r = 0; r < shape.P; ++r) p.dest[r] = dest[r];
+  p.spans = spans;
+  return launched(xs::launch_attention(p, xs::kSeqScatterSpans, reinterpret_cast<cudaStream_t>(stream)),
+                  "attention launch");
+}
+
 xs_status xs_attn_a2a_fused_rank(const void *q, const void *k, const void *v, void *const *dest,
                                  xs_shape shape, int heads_total, int head_offset, float scale,
                                  xs_stream_t stream, int *dev_status) {

@@ -467,12 +467,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       if (!ok) break;
       ++item_cnt;
       ptx::tc_fence_after();
+      // Store-issue span of this warp's share of the tile (kSeqScatterSpans): SM clock before
+      // its first store is prepared and after its last store is issued, and the global timer.
+      [[maybe_unused]] unsigned long long span_clk0 = 0, span_ns0 = 0;
+      if constexpr (EPI == kSeqScatterSpans) {
+        span_clk0 = clock64();
+        span_ns0 = ptx::globaltimer();
+      }
       const float inv_l = 1.f / l_run;
       // Destination of this thread's row.
       const int s_row = q0 + 128 * t + row;
       uint8_t *dst_row = nullptr;
       if (s_row < p.S) {
-        if constexpr (EPI == kSeqScatter) {
+        if constexpr (EPI == kSeqScatter || EPI == kSeqScatterSpans) {
           const int b = bh / p.H;
           const int h = bh - b * p.H + p.head_offset;  // global head index
           const int r = s_row / p.S_local;
@@ -548,6 +555,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         }
         __syncwarp();
       }
+      if constexpr (EPI == kSeqScatterSpans) {
+        // The stores above are only issued, not complete: this is the sender-visible time.
+        const unsigned long long clk1 = clock64();
+        if (lane == 0) {
+          unsigned long long *sp = p.spans + ((static_cast<size_t>(item) * 2 + t) * 4 + wq) * 3;
+          sp[0] = span_clk0;
+          sp[1] = clk1;
+          sp[2] = span_ns0;
+        }
+      }
     }
   }
 
@@ -588,6 +605,8 @@ size_t attention_smem_bytes(int dch) { return dch == 1 ? Smem<1>::kAlloc : Smem<
 
 cudaError_t launch_attention(const AttnParams &p, int epilogue, cudaStream_t stream) {
   const int dch = p.D <= 64 ? 1 : 2;
+  if (epilogue == kSeqScatterSpans)
+    return dch == 1 ? launch_impl<1, kSeqScatterSpans>(p, stream) : launch_impl<2, kSeqScatterSpans>(p, stream);
   if (dch == 1)
     return epilogue == kHeadMajor  ? launch_impl<1, kHeadMajor>(p, stream)
            : epilogue == kPartial ? launch_impl<1, kPartial>(p, stream)

@@ -61,6 +61,7 @@ enum EpilogueKind : int {
   kHeadMajor = 0,   // out[b, h, s, :]
   kSeqScatter = 1,  // dest[r][b, s_local, h, :]  (fused post-attention All-to-All)
   kPartial = 2,     // out[b, h, s, :] in fp32 plus lse[b, h, s] (partial attention of a shard)
+  kSeqScatterSpans = 3,  // kSeqScatter, recording each tile's store-issue span in spans[]
 };
 
 struct AttnParams {
@@ -69,6 +70,7 @@ struct AttnParams {
   CUtensorMap tm_v;
   void *out;               // kHeadMajor (bf16), kPartial (fp32)
   float *lse;              // kPartial: natural-log log-sum-exp of each query row
+  unsigned long long *spans;  // kSeqScatterSpans: [n_items][2 tiles][4 warps][3]
   void *dest[kMaxRanks];   // kSeqScatter
   int B, H, S, D, P;       // H = heads held by this call (the rank's heads); S = query rows
   int S_kv;                // key/value rows (= S except for partial attention over a shard)
