@@ -43,8 +43,8 @@ namespace {
 
 constexpr int kThreads = 320;
 constexpr int kStages = 3;           // K/V ring slots
+constexpr int kStageRows = 16;       // rows staged per warp per epilogue round (head-major / partial)
 constexpr int kChunkBytes = 16384;   // 128 rows x 128 bytes (64 bf16) per swizzle panel
-constexpr int kStageRows = 16;       // rows staged per warp per epilogue round
 constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest tolerated P before rescale
 
 // TMEM column of S_t / P_t and of O_t for Q tile t.
@@ -322,7 +322,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const uint32_t tO = tmem + lane_base + col_o(t);
     const float sl2 = p.scale_log2;
     const int D = p.D;
-    const int nch = D >> 3;          // 16-byte chunks per output row
     uint8_t *stg = base + L::kStage + warp * (kStageRows * L::kStageRowBytes);
     uint8_t **rowptr = reinterpret_cast<uint8_t **>(base + L::kRowPtr) + warp * kStageRows;
     uint32_t sc = 0;       // s_full phases consumed
@@ -497,36 +496,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           p.lse[static_cast<size_t>(bh) * p.S + s_row] = (m_run + log2f(l_run)) * 0.69314718055994531f;
         }
       }
-      // Rounds of kRows rows per warp (16 in bf16, 8 in fp32): stage rows in shared memory
-      // (chunk order rotated by row to spread banks), then write whole rows with consecutive
-      // lanes on consecutive 16-byte chunks.  The stores are not waited for: the warp goes
-      // straight on to its next tile while they drain.
-      // O is read from TMEM once per round, 32 columns at a time (the warp-collective load
-      // brings all 32 rows; the lanes of the current round keep theirs).
-      constexpr int kEB = EPI == kPartial ? 4 : 2;        // bytes per output element
-      constexpr int kRows = kStageRows * 2 / kEB;          // rows per round
-      constexpr int kRowBytes = L::kStageRowBytes * kEB / 2;
-      constexpr int kChunksPerLd = 2 * kEB;                // 16-byte chunks per 32 columns
-      const int nch = D * kEB / 16;                        // 16-byte chunks per output row
-#pragma unroll
-      for (int rd = 0; rd < 32 / kRows; ++rd) {
-        const bool mine = lane / kRows == rd;
-        const int rr = lane % kRows;
-        const int rot = rr % nch;
-        uint8_t *my = stg + rr * kRowBytes;
+      if constexpr (EPI == kSeqScatter || EPI == kSeqScatterSpans) {
+        // Exchange epilogue: each thread writes its own row straight from the TMEM load, 16
+        // bytes at a time, in order along the row.  No staging in shared memory: while the
+        // next item's Q K^T MMAs read both operands from shared memory, staged stores took
+        // several times longer to issue (per-tile store-issue span 5.5 us staged, 3.9 us
+        // direct).  The stores are not waited for: the warp goes straight on to its next tile
+        // while they drain.
+        constexpr int kEB = EPI == kPartial ? 4 : 2;        // bytes per output element
+        constexpr int kChunksPerLd = 2 * kEB;                // 16-byte chunks per 32 columns
+        const int nch = D * kEB / 16;                        // 16-byte chunks per output row
 #pragma unroll
         for (int cc = 0; cc < DCH * 2; ++cc) {
           uint32_t o[32];
           ptx::tmem_ld32(tO + cc * 32, o);
           ptx::tmem_wait_ld();
           ptx::reg_fence32(o);
-          if (mine) {
+          if (dst_row != nullptr) {
 #pragma unroll
             for (int q4 = 0; q4 < kChunksPerLd; ++q4) {
               const int c = cc * kChunksPerLd + q4;  // 16-byte chunk of the output row
               if (c < nch) {
-                int pc = c + rot;
-                if (pc >= nch) pc -= nch;
                 uint32_t w[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -535,25 +525,72 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                   else
                     w[i] = f2u(u2f(o[4 * q4 + i]) * inv_l);
                 }
-                *reinterpret_cast<uint4 *>(my + pc * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+                ptx::st_global_v4(dst_row + c * 16, make_uint4(w[0], w[1], w[2], w[3]));
               }
             }
           }
         }
-        if (mine) rowptr[rr] = dst_row;
-        __syncwarp();
-        for (int idx = lane; idx < kRows * nch; idx += 32) {
-          const int r2 = idx / nch;
-          const int c = idx - r2 * nch;
-          uint8_t *dr = rowptr[r2];
-          if (dr != nullptr) {
-            int pc = c + r2 % nch;
-            if (pc >= nch) pc -= nch;
-            const uint4 v = *reinterpret_cast<const uint4 *>(stg + r2 * kRowBytes + pc * 16);
-            ptx::st_global_v4(dr + c * 16, v);
+      } else {
+        // Head-major and partial epilogues: rounds of kRows rows per warp (16 in bf16, 8 in
+        // fp32) staged in shared memory (chunk order rotated by row to spread banks), then
+        // whole rows written with consecutive lanes on consecutive 16-byte chunks (storing
+        // each thread's row directly made the L2 read the partly written sectors of these
+        // contiguous rows back from DRAM: +1.1 bytes read per byte written).  The stores are not waited for: the warp goes
+        // straight on to its next tile while they drain.
+        // O is read from TMEM once per round, 32 columns at a time (the warp-collective load
+        // brings all 32 rows; the lanes of the current round keep theirs).
+        constexpr int kEB = EPI == kPartial ? 4 : 2;        // bytes per output element
+        constexpr int kRows = kStageRows * 2 / kEB;          // rows per round
+        constexpr int kRowBytes = L::kStageRowBytes * kEB / 2;
+        constexpr int kChunksPerLd = 2 * kEB;                // 16-byte chunks per 32 columns
+        const int nch = D * kEB / 16;                        // 16-byte chunks per output row
+#pragma unroll
+        for (int rd = 0; rd < 32 / kRows; ++rd) {
+          const bool mine = lane / kRows == rd;
+          const int rr = lane % kRows;
+          const int rot = rr % nch;
+          uint8_t *my = stg + rr * kRowBytes;
+#pragma unroll
+          for (int cc = 0; cc < DCH * 2; ++cc) {
+            uint32_t o[32];
+            ptx::tmem_ld32(tO + cc * 32, o);
+            ptx::tmem_wait_ld();
+            ptx::reg_fence32(o);
+            if (mine) {
+#pragma unroll
+              for (int q4 = 0; q4 < kChunksPerLd; ++q4) {
+                const int c = cc * kChunksPerLd + q4;  // 16-byte chunk of the output row
+                if (c < nch) {
+                  int pc = c + rot;
+                  if (pc >= nch) pc -= nch;
+                  uint32_t w[4];
+#pragma unroll
+                  for (int i = 0; i < 4; ++i) {
+                    if constexpr (kEB == 2)
+                      w[i] = ptx::pack_bf16(u2f(o[8 * q4 + 2 * i]) * inv_l, u2f(o[8 * q4 + 2 * i + 1]) * inv_l);
+                    else
+                      w[i] = f2u(u2f(o[4 * q4 + i]) * inv_l);
+                  }
+                  *reinterpret_cast<uint4 *>(my + pc * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+              }
+            }
           }
+          if (mine) rowptr[rr] = dst_row;
+          __syncwarp();
+          for (int idx = lane; idx < kRows * nch; idx += 32) {
+            const int r2 = idx / nch;
+            const int c = idx - r2 * nch;
+            uint8_t *dr = rowptr[r2];
+            if (dr != nullptr) {
+              int pc = c + r2 % nch;
+              if (pc >= nch) pc -= nch;
+              const uint4 v = *reinterpret_cast<const uint4 *>(stg + r2 * kRowBytes + pc * 16);
+              ptx::st_global_v4(dr + c * 16, v);
+            }
+          }
+          __syncwarp();
         }
-        __syncwarp();
       }
       if constexpr (EPI == kSeqScatterSpans) {
         // The stores above are only issued, not complete: this is the sender-visible time.
