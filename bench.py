@@ -7,9 +7,10 @@ line on rank 0:
 
 * ``value``     -- TFLOP/s (4*B*H*S^2*D per step and rank, summed over ranks, divided by the
                    max over ranks of the device time of the K timed steps);
-* ``e2e``       -- the same metric through the public API with host buffers: per step, pinned
-                   host -> device copies of Q, K, V, the fused call, device -> host copies of
-                   the P slabs;
+* ``e2e``       -- the same metric through the public API with host buffers
+                   (``HostPipeline``): per step, pinned host -> device copies of Q, K, V, the
+                   fused calls, device -> host copies of the P slabs, with the heads in groups
+                   whose copies overlap the other groups' kernels;
 * ``roofline``  -- the fused kernel against the measured dense bf16 tensor peak;
 * ``serial_ms`` / ``attn_only_ms`` / ``relayout_ms`` -- attention then the separate exchange
                    pass, attention alone, and the exchange alone, timed the same way;
@@ -353,7 +354,7 @@ def run_xs(args):
             raise RuntimeError("device status non-zero in the end-to-end run")
         e2e = {"value": flops * world / (e2e_ms / n_e2e / 1e3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": pipe.h2d_bytes, "d2h_bytes_per_step": pipe.d2h_bytes,
-               "ms_per_step": e2e_ms / n_e2e}
+               "ms_per_step": e2e_ms / n_e2e, "head_groups": len(pipe.groups)}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -362,25 +362,51 @@ def alloc_dest(B: int, H: int, S: int, D: int, P: int, device=None, fill: float 
 class HostPipeline:
     """End-to-end call with host buffers: pinned host q/k/v in, pinned host slabs out.
 
-    ``run`` enqueues on one stream: three host-to-device copies, the fused kernel, and one
-    device-to-host copy per slab.  Device buffers are allocated once, here, by PyTorch.
+    The heads are split into ``chunks`` groups that flow through three streams: host-to-device
+    copies of a group's q, k, v (input-copy stream), the fused per-rank call for that group's
+    heads writing every slab at the group's head offset (the caller's stream), and
+    device-to-host copies of those heads' columns of every slab (output-copy stream, one
+    2-D copy per slab).  The copies of one group overlap the kernels of the others; events
+    order each group's stages and, across calls, the reuse of its buffers.  ``run`` makes the
+    caller's stream wait for every copy it started, so work timed on that stream covers the
+    whole step.  ``chunks=1`` runs copies, kernel and copies in sequence on the caller's stream.
+    Device buffers are allocated once, here, by PyTorch.
     """
 
-    def __init__(self, B: int, H: int, S: int, D: int, P: int, device=None, scale=None):
+    def __init__(self, B: int, H: int, S: int, D: int, P: int, device=None, scale=None,
+                 chunks: int | None = None):
         import torch
         self.shape = (B, H, S, D)
         self.P = P
         self.scale = scale
         dev = device or torch.device("cuda")
-        self.q = torch.empty(self.shape, dtype=torch.bfloat16, device=dev)
-        self.k = torch.empty_like(self.q)
-        self.v = torch.empty_like(self.q)
+        self.device = dev
+        if chunks is None:
+            # about one wave of 256-row work items per group, at most 20 groups (on the video
+            # workload 20 groups gave 24.2 ms per step, 8 gave 25.4, 4 gave 26.0, 1 gave 43.0)
+            sms = torch.cuda.get_device_properties(dev).multi_processor_count
+            items_per_head = B * ((S + 255) // 256)
+            chunks = max(1, min(20, H, (H * items_per_head) // sms))
+        self.chunks = int(chunks)
+        hc = (H + self.chunks - 1) // self.chunks
+        self.groups = [(h0, min(H, h0 + hc)) for h0 in range(0, H, hc)]
+        # per-group contiguous device inputs [B, Hc, S, D]
+        self.q = [torch.empty((B, h1 - h0, S, D), dtype=torch.bfloat16, device=dev) for h0, h1 in self.groups]
+        self.k = [torch.empty_like(t) for t in self.q]
+        self.v = [torch.empty_like(t) for t in self.q]
         self.dest = alloc_dest(B, H, S, D, P, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.s_in = torch.cuda.Stream(device=dev)
+        self.s_out = torch.cuda.Stream(device=dev)
+        n = len(self.groups)
+        self.ev_in = [torch.cuda.Event() for _ in range(n)]     # group's inputs on the device
+        self.ev_kern = [torch.cuda.Event() for _ in range(n)]   # group's kernel done
+        self.ev_out = [torch.cuda.Event() for _ in range(n)]    # group's columns copied out
+        self._started = False
 
     @property
     def h2d_bytes(self) -> int:
-        return 3 * self.q.numel() * 2
+        return 3 * sum(t.numel() for t in self.q) * 2
 
     @property
     def d2h_bytes(self) -> int:
@@ -388,12 +414,43 @@ class HostPipeline:
 
     def run(self, q_host, k_host, v_host, dest_host, stream=None):
         import torch
+        from cuda.bindings import runtime as rt
         s = stream or torch.cuda.current_stream()
-        with torch.cuda.stream(s):
-            self.q.copy_(q_host, non_blocking=True)
-            self.k.copy_(k_host, non_blocking=True)
-            self.v.copy_(v_host, non_blocking=True)
-            attn_a2a_fused(self.q, self.k, self.v, self.dest, scale=self.scale, stream=s,
-                           status=self.status)
+        B, H, S, D = self.shape
+        Sl = S // self.P
+        row_bytes = H * D * 2
+        start = torch.cuda.Event()
+        start.record(s)
+        self.s_in.wait_event(start)
+        self.s_out.wait_event(start)
+        for g, (h0, h1) in enumerate(self.groups):
+            # inputs: the group's buffers are free once its previous kernel is done
+            with torch.cuda.stream(self.s_in):
+                if self._started:
+                    self.s_in.wait_event(self.ev_kern[g])
+                for b in range(B):
+                    self.q[g][b].copy_(q_host[b, h0:h1], non_blocking=True)
+                    self.k[g][b].copy_(k_host[b, h0:h1], non_blocking=True)
+                    self.v[g][b].copy_(v_host[b, h0:h1], non_blocking=True)
+                self.ev_in[g].record(self.s_in)
+            # kernel: its inputs have landed and its slab columns have been copied out
+            s.wait_event(self.ev_in[g])
+            if self._started:
+                s.wait_event(self.ev_out[g])
+            attn_a2a_fused_rank(self.q[g], self.k[g], self.v[g], self.dest, heads_total=H,
+                                head_offset=h0, scale=self.scale, stream=s, status=self.status)
+            self.ev_kern[g].record(s)
+            # outputs: the group's heads in every slab, one 2-D copy per slab
+            self.s_out.wait_event(self.ev_kern[g])
+            width = (h1 - h0) * D * 2
             for dh, dd in zip(dest_host, self.dest):
-                dh.copy_(dd, non_blocking=True)
+                err, = rt.cudaMemcpy2DAsync(dh.data_ptr() + h0 * D * 2, row_bytes, dd.data_ptr() + h0 * D * 2,
+                                            row_bytes, width, B * Sl,
+                                            rt.cudaMemcpyKind.cudaMemcpyDeviceToHost, self.s_out.cuda_stream)
+                if err != rt.cudaError_t.cudaSuccess:
+                    raise RuntimeError(f"output copy failed: {err}")
+            self.ev_out[g].record(self.s_out)
+        self._started = True
+        # the caller's stream covers every copy of this step
+        for g in range(len(self.groups)):
+            s.wait_event(self.ev_out[g])
