@@ -413,10 +413,24 @@ class HostPipeline:
         return sum(d.numel() * 2 for d in self.dest)
 
     def run(self, q_host, k_host, v_host, dest_host, stream=None):
+        """Enqueue one step: ``q_host, k_host, v_host`` pinned CPU bf16 [B, H, S, D] in,
+        ``dest_host`` P pinned CPU bf16 slabs [B, S/P, H, D] out (ready after the caller's
+        stream has reached the point where ``run`` returned)."""
         import torch
         from cuda.bindings import runtime as rt
         s = stream or torch.cuda.current_stream()
         B, H, S, D = self.shape
+        for name, t in (("q_host", q_host), ("k_host", k_host), ("v_host", v_host)):
+            if tuple(t.shape) != self.shape or t.dtype != torch.bfloat16 or t.is_cuda \
+                    or not t.is_contiguous() or not t.is_pinned():
+                raise ValueError(f"{name} must be a contiguous pinned CPU bf16 tensor of shape {self.shape}")
+        if len(dest_host) != self.P:
+            raise ValueError(f"need {self.P} host slabs, got {len(dest_host)}")
+        for r, t in enumerate(dest_host):
+            if tuple(t.shape) != tuple(self.dest[r].shape) or t.dtype != torch.bfloat16 or t.is_cuda \
+                    or not t.is_contiguous() or not t.is_pinned():
+                raise ValueError(f"dest_host[{r}] must be a contiguous pinned CPU bf16 tensor of shape "
+                                 f"{tuple(self.dest[r].shape)}")
         Sl = S // self.P
         row_bytes = H * D * 2
         start = torch.cuda.Event()
