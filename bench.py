@@ -14,10 +14,19 @@ line on rank 0:
 * ``roofline``  -- the fused kernel against the measured dense bf16 tensor peak;
 * ``serial_ms`` / ``attn_only_ms`` / ``relayout_ms`` -- attention then the separate exchange
                    pass, attention alone, and the exchange alone, timed the same way;
+                   ``fused_vs_serial`` and ``fused_vs_attn_only`` are time ratios (fused time
+                   divided by the other; below 1 means the fused step is faster);
 * ``cpu_baseline`` -- the CPU oracle (fp64, OpenMP) on a bounded sample of the same workload.
 
 ``--impl reference`` times that CPU oracle alone (rank 0 only) on the same workload.
-``--gpus N`` under torchrun runs N independent replicas (one per GPU): weak scaling.
+``--gpus N`` under torchrun (N > 1, NCCL) runs one Ulysses layer of the workload over the N GPUs
+(strong scaling): GPU g computes heads [g*H/N, (g+1)*H/N) and holds the slabs of ranks
+[g*P/N, (g+1)*P/N); its fused call stores every finished tile into the slab of the rank
+that needs it, on whichever GPU that is (CUDA IPC mappings, NVLink stores), and a
+one-element all-reduce after it orders those stores (``multigpu.UlyssesGpu``).  The serial
+step is attention, a pack by the exchange kernel, an NCCL all-to-all and an unpack.
+When a GPU's Q, K and V fit in L2, every timed step is preceded by a read of a buffer twice
+the L2 size, outside the step's events.
 """
 from __future__ import annotations
 
@@ -51,6 +60,10 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU-oracle sample time")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--dist-backend", choices=["nccl", "gloo"], default="nccl",
+                    help="process group for N > 1; gloo orders the GPUs through the host and lets "
+                         "several processes share one GPU: a check of the multi-process path, not a "
+                         "measurement")
     return ap.parse_args(argv)
 
 
@@ -65,7 +78,7 @@ def reduce_max(x: float, device=None) -> float:
     import torch.distributed as dist
     if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device=device)
+    t = torch.tensor([x], dtype=torch.float64, device=device if dist.get_backend() == "nccl" else "cpu")
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -73,7 +86,7 @@ def reduce_max(x: float, device=None) -> float:
 def barrier(device=None):
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
-        if device is not None and device.type == "cuda":
+        if device is not None and device.type == "cuda" and dist.get_backend() == "nccl":
             dist.barrier(device_ids=[device.index])
         else:
             dist.barrier()
@@ -89,14 +102,18 @@ def measured_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+# The sources that define the attention kernel and its launch (tensor maps, parameters).
+KERNEL_SOURCES = ("api.cu", "attn.cu", "ptx.cuh", "xs_internal.cuh")
+
+
 def source_digest() -> str:
-    """Hash of the CUDA sources: a profile summary is only valid for the kernel it measured."""
+    """Hash of the attention kernel's sources: a profile summary is only valid for the kernel
+    it measured."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "ulysses_attention_output_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, fn), "rb") as f:
-                h.update(fn.encode() + b"\0" + f.read())
+    for fn in KERNEL_SOURCES:
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
@@ -179,24 +196,50 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def time_steps(fn, steps: int, warmup: int, stream, device):
-    """Device time (ms) of `steps` back-to-back calls of fn() on `stream`, max over ranks."""
+def time_steps(fn, steps: int, warmup: int, stream, device, flush=None):
+    """Device time (ms) of `steps` calls of fn() on `stream`, max over ranks.
+
+    Without `flush`: one event pair around the back-to-back calls (inputs larger than L2).
+    With `flush` (a uint8 device buffer larger than L2): before every call the buffer is
+    read on `stream` outside the timed region, so each call starts with no line of its
+    inputs in L2; the result is the sum of the calls' own event-pair times."""
     import torch
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize(device)
     barrier(device)
     torch.cuda.synchronize(device)
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    for _ in range(steps):
-        fn()
-    ev1.record(stream)
+    if flush is None:
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(steps):
+            fn()
+        ev1.record(stream)
+        pairs = [(ev0, ev1)]
+    else:
+        sink = torch.zeros((), dtype=torch.int32, device=device)
+        words = flush.view(torch.int32)
+        pairs = []
+        for _ in range(steps):
+            sink.copy_(words.amax())
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            pairs.append((e0, e1))
     torch.cuda.synchronize(device)
     barrier(device)
     torch.cuda.synchronize(device)
-    return reduce_max(ev0.elapsed_time(ev1), device)
+    return reduce_max(sum(e0.elapsed_time(e1) for e0, e1 in pairs), device)
+
+
+def l2_flush_buffer(input_bytes: int, device):
+    """A buffer twice the L2 size when the inputs fit in L2, else None (no flush needed)."""
+    import torch
+    if input_bytes > L2_BYTES:
+        return None
+    return torch.zeros(2 * L2_BYTES, dtype=torch.uint8, device=device)
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -249,11 +292,14 @@ def oracle_sample(w, target_s: float):
 
 
 # ----------------------------------------------------------------------------- arms
-def workload_config(w):
+def workload_config(w, world: int = 1):
+    per_gpu = w.qkv_bytes // world
     return {"workload": w.name, "description": w.description, "B": w.B, "H": w.H, "S": w.S,
             "D": w.D, "P": w.P, "structure": w.structure,
-            "l2": (f"inputs larger than L2 ({w.qkv_bytes / 2**20:.0f} MiB > 126 MiB), no flush"
-                   if w.qkv_bytes > L2_BYTES else "L2 flushed between steps")}
+            "l2": (f"inputs per GPU larger than L2 ({per_gpu / 2**20:.0f} MiB > 126 MiB), no flush"
+                   if per_gpu > L2_BYTES else
+                   f"inputs per GPU {per_gpu / 2**20:.0f} MiB fit in L2: a 252 MiB buffer is read "
+                   f"before every timed step, outside its events")}
 
 
 def run_reference(args):
@@ -285,99 +331,192 @@ def run_reference(args):
     return 0
 
 
+class SingleGpu:
+    """One GPU holds every head and all P slabs: the fused call, its parts and the e2e path."""
+
+    def __init__(self, w, device, stream):
+        import torch
+
+        import ulysses_attention_output_b200 as xs
+        from ulysses_attention_output_b200 import workloads as W
+        self.xs, self.w, self.device, self.stream = xs, w, device, stream
+        self.q_h, self.k_h, self.v_h = W.make_inputs(w)
+        self.q, self.k, self.v = (t.to(device) for t in (self.q_h, self.k_h, self.v_h))
+        self.dest = xs.alloc_dest(w.B, w.H, w.S, w.D, w.P, device=device)
+        self.out = torch.empty_like(self.q)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.flops_gpu = xs.attention_flops(w.B, w.H, w.S, w.D)
+        self.input_bytes = w.qkv_bytes
+
+    def fused(self):
+        self.xs.attn_a2a_fused(self.q, self.k, self.v, self.dest, stream=self.stream, status=self.status)
+
+    def attn_only(self):
+        self.xs.attn(self.q, self.k, self.v, self.out, stream=self.stream, status=self.status)
+
+    def relayout(self):
+        self.xs.a2a_relayout(self.out, self.dest, stream=self.stream)
+
+    def serial(self):
+        self.attn_only()
+        self.relayout()
+
+    def e2e(self):
+        """(step function, status tensor, h2d bytes, d2h bytes, extras) through HostPipeline."""
+        import torch
+        w = self.w
+        pipe = self.xs.HostPipeline(w.B, w.H, w.S, w.D, w.P, device=self.device)
+        qp, kp, vp = (t.pin_memory() for t in (self.q_h, self.k_h, self.v_h))
+        dest_h = [torch.empty(d.shape, dtype=d.dtype).pin_memory() for d in pipe.dest]
+        return (lambda: pipe.run(qp, kp, vp, dest_h, stream=self.stream), pipe.status,
+                pipe.h2d_bytes, pipe.d2h_bytes, {"head_groups": len(pipe.groups)})
+
+    def close(self):
+        pass
+
+
+class UlyssesGpus:
+    """One of N GPUs of a Ulysses layer (NCCL): this GPU's H/N heads; its P/N slabs, which the
+    other GPUs' fused calls store into through CUDA IPC mappings over NVLink."""
+
+    def __init__(self, w, device, stream):
+        import torch
+
+        import ulysses_attention_output_b200 as xs
+        from ulysses_attention_output_b200 import multigpu as MG
+        from ulysses_attention_output_b200 import workloads as W
+        self.xs, self.w, self.device, self.stream = xs, w, device, stream
+        self.layer = MG.UlyssesGpu(w.B, w.H, w.S, w.D, w.P, device=device)
+        pl = self.plan = self.layer.plan
+        hs = slice(pl.head_offset, pl.head_offset + pl.heads_local)
+        self.q_h, self.k_h, self.v_h = (t[:, hs].contiguous() for t in W.make_inputs(w))
+        self.q, self.k, self.v = (t.to(device) for t in (self.q_h, self.k_h, self.v_h))
+        self.out, self.send, self.recv = self.layer.alloc_exchange_buffers()
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.flops_gpu = xs.attention_flops(w.B, pl.heads_local, w.S, w.D)
+        self.input_bytes = 3 * self.q.numel() * 2
+
+    def fused(self):
+        self.layer.fused(self.q, self.k, self.v, stream=self.stream, status=self.status)
+        self.layer.complete(self.stream)
+
+    def attn_only(self):
+        self.xs.attn(self.q, self.k, self.v, self.out, stream=self.stream, status=self.status)
+
+    def relayout(self):
+        self.xs.a2a_relayout(self.out, [self.send[r] for r in range(self.w.P)], stream=self.stream)
+        self.layer.exchange_packed(self.send, self.recv, stream=self.stream)
+
+    def serial(self):
+        self.attn_only()
+        self.relayout()
+
+    def e2e(self):
+        """Per step: this GPU's Q, K, V from pinned host memory, the fused call, completion,
+        its slabs back to pinned host memory, and a second completion so that no GPU's next
+        fused call overwrites a slab that is still being copied out."""
+        import torch
+        qp, kp, vp = (t.pin_memory() for t in (self.q_h, self.k_h, self.v_h))
+        slabs_h = torch.empty(self.layer.slabs.shape, dtype=torch.bfloat16).pin_memory()
+
+        def step():
+            for dev_t, host_t in ((self.q, qp), (self.k, kp), (self.v, vp)):
+                dev_t.copy_(host_t, non_blocking=True)
+            self.fused()
+            slabs_h.copy_(self.layer.slabs, non_blocking=True)
+            self.layer.complete(self.stream)
+        h2d = 3 * self.q.numel() * 2
+        return step, self.status, h2d, slabs_h.numel() * 2, {"overlap": "none (copies, kernel, copies in sequence)"}
+
+    def close(self):
+        self.layer.close()
+
+
 def run_xs(args):
     import torch
     import torch.distributed as dist
 
-    import ulysses_attention_output_b200 as xs
     from ulysses_attention_output_b200 import workloads as W
 
     rank, local_rank, world = dist_env()
-    torch.cuda.set_device(local_rank)
-    device = torch.device("cuda", local_rank)
+    # gloo may put several processes on one GPU; with NCCL every process has its own GPU
+    dev_index = local_rank if args.dist_backend == "nccl" else local_rank % torch.cuda.device_count()
+    torch.cuda.set_device(dev_index)
+    device = torch.device("cuda", dev_index)
     if world > 1 and not dist.is_initialized():
         from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+        if args.dist_backend == "nccl":
+            dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+        else:
+            dist.init_process_group("gloo", timeout=timedelta(seconds=120))
+    import ulysses_attention_output_b200 as xs
     xs.load()
     w = W.WORKLOADS[args.workload]
-    B, H, S, D, P = w.B, w.H, w.S, w.D, w.P
-    q_h, k_h, v_h = W.make_inputs(w)
-    q, k, v = (t.to(device) for t in (q_h, k_h, v_h))
-    dest = xs.alloc_dest(B, H, S, D, P, device=device)
-    out = torch.empty_like(q)
-    status = torch.zeros(1, dtype=torch.int32, device=device)
     stream = torch.cuda.Stream(device)
-    flops = xs.attention_flops(B, H, S, D)
-
-    def fused():
-        xs.attn_a2a_fused(q, k, v, dest, stream=stream, status=status)
-
-    def attn_only():
-        xs.attn(q, k, v, out, stream=stream, status=status)
-
-    def relayout():
-        xs.a2a_relayout(out, dest, stream=stream)
-
-    def serial():
-        attn_only()
-        relayout()
+    g = (UlyssesGpus if world > 1 else SingleGpu)(w, device, stream)
+    flush = l2_flush_buffer(g.input_bytes, device)
 
     with torch.cuda.stream(stream):
         with ClockSampler(device.index) as clk:
-            fused_ms = time_steps(fused, args.steps, args.warmup, stream, device)
-        attn_ms = time_steps(attn_only, args.steps, args.warmup, stream, device)
-        relayout_ms = time_steps(relayout, args.steps, args.warmup, stream, device)
-        serial_ms = time_steps(serial, args.steps, args.warmup, stream, device)
+            fused_ms = time_steps(g.fused, args.steps, args.warmup, stream, device, flush)
+        attn_ms = time_steps(g.attn_only, args.steps, args.warmup, stream, device, flush)
+        relayout_ms = time_steps(g.relayout, args.steps, args.warmup, stream, device, flush)
+        serial_ms = time_steps(g.serial, args.steps, args.warmup, stream, device, flush)
     torch.cuda.synchronize(device)
-    if int(status.item()) != 0:
-        raise RuntimeError(f"device status {int(status.item())} after the timed runs")
+    if int(g.status.item()) != 0:
+        raise RuntimeError(f"device status {int(g.status.item())} after the timed runs")
 
+    flops_job = xs.attention_flops(w.B, w.H, w.S, w.D)   # the whole layer, all GPUs together
     ms_per_step = fused_ms / args.steps
-    value = flops * world / (ms_per_step / 1e3) / 1e12
+    value = flops_job / (ms_per_step / 1e3) / 1e12
     peaks, peak_src = measured_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-    achieved = flops / (ms_per_step / 1e3) / 1e12  # one launch per step on this rank
+    achieved = g.flops_gpu / (ms_per_step / 1e3) / 1e12  # this GPU's launch per step
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    relayout_gbs = 2 * w.out_bytes / (relayout_ms / args.steps / 1e3) / 1e9
+    relayout_gbs = 2 * (w.out_bytes // world) / (relayout_ms / args.steps / 1e3) / 1e9
 
     e2e = None
     if not args.no_e2e:
-        pipe = xs.HostPipeline(B, H, S, D, P, device=device)
-        qp, kp, vp = (t.pin_memory() for t in (q_h, k_h, v_h))
-        dest_h = [torch.empty(d.shape, dtype=d.dtype).pin_memory() for d in pipe.dest]
-        with torch.cuda.stream(stream):
-            e2e_ms = time_steps(lambda: pipe.run(qp, kp, vp, dest_h, stream=stream),
-                                max(3, args.steps // 3), max(3, args.warmup), stream, device)
+        step, st, h2d, d2h, extra = g.e2e()
         n_e2e = max(3, args.steps // 3)
-        if int(pipe.status.item()) != 0:
+        with torch.cuda.stream(stream):
+            e2e_ms = time_steps(step, n_e2e, max(3, args.warmup), stream, device)
+        if int(st.item()) != 0:
             raise RuntimeError("device status non-zero in the end-to-end run")
-        e2e = {"value": flops * world / (e2e_ms / n_e2e / 1e3) / 1e12, "unit": UNIT,
-               "h2d_bytes_per_step": pipe.h2d_bytes, "d2h_bytes_per_step": pipe.d2h_bytes,
-               "ms_per_step": e2e_ms / n_e2e, "head_groups": len(pipe.groups)}
+        e2e = {"value": flops_job / (e2e_ms / n_e2e / 1e3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": h2d * world, "d2h_bytes_per_step": d2h * world,
+               "ms_per_step": e2e_ms / n_e2e, **extra}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cv, threads, desc = oracle_sample(w, args.cpu_seconds)
         cpu = {"value": cv, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
 
+    traffic = profiled_traffic(w.name) if world == 1 else None
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {**workload_config(w), "parallelism": f"replicas{world}" if world > 1 else "single"},
+        "scaling": "strong" if world > 1 else "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {**workload_config(w, world),
+                   "parallelism": f"ulysses{world} (heads {w.H // world} per GPU, NVLink peer stores)"
+                   if world > 1 else "single",
+                   **({"dist_backend": "gloo (host-ordered check, not a measurement)"}
+                      if world > 1 and args.dist_backend == "gloo" else {})},
         "frac_of_bf16_peak": achieved / peak,
         "serial_ms": serial_ms / args.steps, "attn_only_ms": attn_ms / args.steps,
         "relayout_ms": relayout_ms / args.steps,
-        "fused_vs_serial": (serial_ms / fused_ms), "fused_vs_attn_only": fused_ms / attn_ms,
+        "fused_vs_serial": fused_ms / serial_ms, "fused_vs_attn_only": fused_ms / attn_ms,
         "relayout_gbs": relayout_gbs, "relayout_frac_hbm": relayout_gbs / hbm,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": profiled_traffic(w.name),
+                     "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{peak_src} bf16 burst", "peak_sustained": peak_sus,
                      "frac_sustained": achieved / peak_sus, "kernel": "attn_fwd_kernel<2,kSeqScatter>"},
         "e2e": e2e, "cpu_baseline": cpu, "clocks": clk.summary(),
         "gpu_launches": args.steps, "impl": "xs",
     }
+    g.close()
     if rank == 0:
         print(json.dumps(line))
     if world > 1:

@@ -126,8 +126,9 @@ XS_API xs_status xs_attn(const void *q, const void *k, const void *v, void *out,
 /*
  * The post-attention All-to-All as a separate pass (second half of the serial baseline):
  *   dest[r][b, s_local, h, :] = src[b, h, r*S/P + s_local, :]
- * src: device [B, H, S, D] 16-bit words; dest: host array of P device slab pointers.  A pure
- * copy: every destination word equals its source word.
+ * src: device [B, H, S, D] 16-bit words; dest: host array of P device slab pointers, each
+ * [B, S/P, H, D].  A pure copy: every destination word equals its source word.  Needs
+ * S % P == 0 but any H (a GPU holding H/N of a layer's heads packs them per rank with it).
  */
 XS_API xs_status xs_a2a_relayout(const void *src, void *const *dest, xs_shape shape,
                           xs_stream_t stream);
@@ -247,6 +248,45 @@ XS_API xs_status xs_burst_probe_static(xs_burst_cfg cfg, unsigned long long *sta
  * to *dev_status (device, required).  The context stays usable afterwards.
  */
 XS_API xs_status xs_selftest_bounded_wait(int *dev_status, long long limit_ns, xs_stream_t stream);
+
+/*
+ * Peer mapping of destination slabs between the processes of one node (one process per
+ * GPU).  In the multi-GPU form of the exchange (X-Stage explainer, "FlashAttention-A2A
+ * (Piggybacking)": the tile's owner sends the finished tile to the rank that needs it), each
+ * GPU holds the sequence-shard slabs of its own ranks; the other GPUs map them with these
+ * calls and pass the mapped pointers in the `dest` array of xs_attn_a2a_fused_rank, whose
+ * epilogue then stores straight into them over NVLink.  Nothing is allocated or freed here
+ * beyond the mapping itself; no call synchronises a stream.
+ */
+#define XS_IPC_HANDLE_BYTES 64
+
+/*
+ * Export the allocation that contains `ptr` for mapping by other processes.
+ *   ptr    : device pointer into memory from cudaMalloc (directly, or through a caching
+ *            allocator built on it) on any device of this process.
+ *   handle : host buffer of XS_IPC_HANDLE_BYTES bytes; receives the CUDA IPC handle of the
+ *            whole allocation (the handle is opaque and valid on this node only).
+ *   offset : host; receives ptr minus the allocation's first byte.
+ * Errors: XS_ERR_INVALID_ARG for a null argument; XS_ERR_CUDA when the driver refuses (the
+ * memory is not a cudaMalloc allocation, e.g. a virtual-memory mapping).  The exporter must
+ * keep the memory alive until every process that opened the handle has closed it.
+ */
+XS_API xs_status xs_ipc_export(const void *ptr, unsigned char *handle, long long *offset);
+
+/*
+ * Map an allocation exported by another process of this node.
+ *   handle : host, XS_IPC_HANDLE_BYTES bytes from xs_ipc_export in that process.
+ *   base   : host; receives the mapped address of the allocation's first byte in this
+ *            process (add the exporter's offset to reach its pointer).  Peer access from the
+ *            current device to the owning device is enabled on first use.
+ * Errors: XS_ERR_INVALID_ARG for a null argument; XS_ERR_CUDA when the driver refuses (the
+ * handle came from this same process, or the devices cannot reach each other).
+ * Every successful open is paired with one xs_ipc_close(base).
+ */
+XS_API xs_status xs_ipc_open(const unsigned char *handle, void **base);
+
+/* Unmap a base returned by xs_ipc_open; no kernel that stores through it may still run. */
+XS_API xs_status xs_ipc_close(void *base);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 XS_API const char *xs_get_error_string(xs_status status);

@@ -87,6 +87,7 @@ def test_attn_and_relayout_reject(lib):
     arr = (ctypes.c_void_p * 2)(FAKE + 100 * MB, FAKE + 200 * MB)
     assert lib.xs_a2a_relayout(0, arr, sh, None) == xs.XS_ERR_INVALID_ARG
     assert lib.xs_a2a_relayout(FAKE, arr, xs.Shape(1, 4, 256, 60, 2), None) == xs.XS_ERR_UNSUPPORTED
+    assert lib.xs_a2a_relayout(FAKE, arr, xs.Shape(1, 4, 250, 64, 4), None) == xs.XS_ERR_UNSUPPORTED  # S % P
 
 
 def test_probe_and_selftest_reject(lib):
@@ -140,3 +141,26 @@ def test_partial_and_merge_reject(lib):
     assert M(op, lp, 2, FAKE + 1024, None, 1024, 128, None) == xs.XS_ERR_INVALID_ARG      # out inside part 0
     bad = (ctypes.c_void_p * 2)(FAKE + 4, FAKE + 4 * MB)
     assert M(bad, lp, 2, out, None, 1024, 128, None) == xs.XS_ERR_INVALID_ARG             # misaligned part
+
+
+def test_ipc_calls_reject_null_arguments(lib):
+    buf = ctypes.create_string_buffer(xs.IPC_HANDLE_BYTES)
+    off = ctypes.c_longlong(0)
+    base = ctypes.c_void_p(0)
+    assert lib.xs_ipc_export(None, buf, ctypes.byref(off)) == xs.XS_ERR_INVALID_ARG
+    assert lib.xs_ipc_export(FAKE, None, ctypes.byref(off)) == xs.XS_ERR_INVALID_ARG
+    assert lib.xs_ipc_export(FAKE, buf, None) == xs.XS_ERR_INVALID_ARG
+    assert lib.xs_ipc_open(None, ctypes.byref(base)) == xs.XS_ERR_INVALID_ARG
+    assert lib.xs_ipc_open(buf, None) == xs.XS_ERR_INVALID_ARG
+    assert lib.xs_ipc_close(None) == xs.XS_ERR_INVALID_ARG
+    assert "non-null" in lib.xs_last_error_detail().decode()
+
+
+def test_ipc_binding_checks_its_arguments():
+    import torch
+    with pytest.raises(ValueError):
+        xs.ipc_export(torch.zeros(4))              # host tensor
+    with pytest.raises(ValueError):
+        xs.ipc_open(b"\0" * (xs.IPC_HANDLE_BYTES - 1))
+    ptr_text = open(os.path.join(ROOT, "include", "xs.h")).read()
+    assert re.search(r"#define XS_IPC_HANDLE_BYTES (\d+)", ptr_text).group(1) == str(xs.IPC_HANDLE_BYTES)

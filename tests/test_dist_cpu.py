@@ -65,3 +65,14 @@ def test_single_process_reduce_is_identity():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.reduce_max(2.5) == 2.5
+
+
+def test_l2_flush_decision_per_gpu():
+    sys.path.insert(0, ROOT)
+    import bench
+    from ulysses_attention_output_b200 import workloads as W
+    video, mmdit = W.WORKLOADS["video"], W.WORKLOADS["mmdit"]
+    assert "no flush" in bench.workload_config(video, 1)["l2"]        # 960 MiB
+    assert "no flush" in bench.workload_config(video, 4)["l2"]        # 240 MiB per GPU
+    assert "before every timed step" in bench.workload_config(video, 8)["l2"]  # 120 MiB per GPU
+    assert "before every timed step" in bench.workload_config(mmdit, 1)["l2"]  # 81 MiB

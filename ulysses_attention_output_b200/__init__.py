@@ -29,10 +29,12 @@ __all__ = [
     "library_path", "load", "version", "attn_a2a_fused", "attn", "a2a_relayout", "burst_probe",
     "attn_a2a_fused_rank", "a2a_pre", "attn_partial", "lse_merge", "attn_a2a_fused_spans",
     "burst_probe_static", "selftest_bounded_wait", "alloc_dest", "HostPipeline", "attention_flops",
+    "ipc_export", "ipc_open", "ipc_close", "IPC_HANDLE_BYTES",
 ]
 
 XS_OK, XS_ERR_INVALID_ARG, XS_ERR_UNSUPPORTED, XS_ERR_CUDA, XS_ERR_TIMEOUT = 0, 1, 2, 3, 4
 XS_MAX_RANKS = 16
+IPC_HANDLE_BYTES = 64  # XS_IPC_HANDLE_BYTES
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _lock = threading.Lock()
@@ -91,6 +93,9 @@ def load():
         lib.xs_attn_partial.argtypes = [vp, vp, vp, vp, vp, Shape, c_int, c_float, vp, ip]
         lib.xs_attn_a2a_fused_spans.argtypes = [vp, vp, vp, vpp, Shape, c_float, vp, ctypes.c_longlong, vp, ip]
         lib.xs_lse_merge.argtypes = [vpp, vpp, c_int, vp, vp, ctypes.c_longlong, c_int, vp]
+        lib.xs_ipc_export.argtypes = [vp, ctypes.c_char_p, ctypes.POINTER(ctypes.c_longlong)]
+        lib.xs_ipc_open.argtypes = [ctypes.c_char_p, ctypes.POINTER(ctypes.c_void_p)]
+        lib.xs_ipc_close.argtypes = [vp]
         for fn in (lib.xs_attn_a2a_fused, lib.xs_attn, lib.xs_a2a_relayout, lib.xs_burst_probe,
                    lib.xs_burst_probe_static, lib.xs_selftest_bounded_wait,
                    lib.xs_attn_a2a_fused_rank, lib.xs_a2a_pre, lib.xs_attn_partial, lib.xs_lse_merge,
@@ -197,17 +202,51 @@ def attn_a2a_fused_spans(q, k, v, dest, spans=None, scale: float | None = None, 
 def attn_a2a_fused_rank(q, k, v, dest, heads_total: int, head_offset: int, scale: float | None = None,
                         stream=None, status=None):
     """One Ulysses rank's fused call: its heads ``q, k, v`` [B, H_rank, S, D] scattered into
-    every rank's slab ``dest[r]`` [B, S/P, heads_total, D] at heads head_offset .. +H_rank."""
+    every rank's slab ``dest[r]`` [B, S/P, heads_total, D] at heads head_offset .. +H_rank.
+
+    An entry of ``dest`` is either a tensor on this GPU or an int: the address of a slab in
+    another process's memory mapped here with ``ipc_open`` (the library checks it for null,
+    alignment and overlap; its extent is the caller's to guarantee)."""
     P = len(dest)
     shp = _shape_of(q, P)
     for n, t in (("q", q), ("k", k), ("v", v)):
         _bf16_cuda(n, t, tuple(q.shape))
+    ptrs = []
     for r, d in enumerate(dest):
-        _bf16_cuda(f"dest[{r}]", d, (shp.B, shp.S // P, int(heads_total), shp.D))
-    arr = (ctypes.c_void_p * P)(*[d.data_ptr() for d in dest])
+        if isinstance(d, int):
+            ptrs.append(d)
+        else:
+            _bf16_cuda(f"dest[{r}]", d, (shp.B, shp.S // P, int(heads_total), shp.D))
+            ptrs.append(d.data_ptr())
+    arr = (ctypes.c_void_p * P)(*ptrs)
     _check(load().xs_attn_a2a_fused_rank(q.data_ptr(), k.data_ptr(), v.data_ptr(), arr, shp,
                                          int(heads_total), int(head_offset), float(scale or 0.0),
                                          _stream_handle(stream), _ptr(status)))
+
+
+def ipc_export(t) -> tuple[bytes, int]:
+    """CUDA IPC handle of the allocation holding tensor ``t`` (on a GPU), and ``t``'s byte
+    offset in it: what another process of this node needs to map ``t`` with ``ipc_open``."""
+    if not getattr(t, "is_cuda", False):
+        raise ValueError("ipc_export needs a CUDA tensor")
+    buf = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    off = ctypes.c_longlong(0)
+    _check(load().xs_ipc_export(t.data_ptr(), buf, ctypes.byref(off)))
+    return buf.raw, int(off.value)
+
+
+def ipc_open(handle: bytes) -> int:
+    """Map an allocation exported by another process; returns its base address here."""
+    if len(handle) != IPC_HANDLE_BYTES:
+        raise ValueError(f"an IPC handle has {IPC_HANDLE_BYTES} bytes, got {len(handle)}")
+    base = ctypes.c_void_p(0)
+    _check(load().xs_ipc_open(handle, ctypes.byref(base)))
+    return int(base.value)
+
+
+def ipc_close(base: int) -> None:
+    """Unmap a base address returned by ``ipc_open``."""
+    _check(load().xs_ipc_close(ctypes.c_void_p(base)))
 
 
 def a2a_pre(src, dst, heads_local: int | None = None, head_offset: int = 0, stream=None):

@@ -12,11 +12,10 @@
 #include "xs.h"
 #include "xs_internal.cuh"
 
-namespace {
-
+namespace xs {
 thread_local char g_detail[512] = "";
 
-xs_status fail(xs_status code, const char *fmt, ...) {
+int record_error(int code, const char *fmt, ...) {
   va_list ap;
   va_start(ap, fmt);
   vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
@@ -24,8 +23,18 @@ xs_status fail(xs_status code, const char *fmt, ...) {
   return code;
 }
 
+void clear_error() { g_detail[0] = '\0'; }
+}  // namespace xs
+
+namespace {
+
+template <typename... A>
+xs_status fail(xs_status code, const char *fmt, A... args) {
+  return static_cast<xs_status>(xs::record_error(code, fmt, args...));
+}
+
 xs_status ok() {
-  g_detail[0] = '\0';
+  xs::clear_error();
   return XS_OK;
 }
 
@@ -346,8 +355,11 @@ xs_status xs_lse_merge(const float *const *o_parts, const float *const *lse_part
 }
 
 xs_status xs_a2a_relayout(const void *src, void *const *dest, xs_shape shape, xs_stream_t stream) {
-  xs_status st = check_shape(shape, true);
+  // Any H: the pack step of a GPU that holds only H/N of the layer's heads uses it too.
+  xs_status st = check_shape(shape, false);
   if (st != XS_OK) return st;
+  if (shape.S % shape.P != 0)
+    return fail(XS_ERR_UNSUPPORTED, "S %% P != 0 (S=%d P=%d)", shape.S, shape.P);
   if (!src || !aligned16(src)) return fail(XS_ERR_INVALID_ARG, "src must be a 16-byte aligned device pointer");
   const void *ins[1] = {src};
   if ((st = check_dest(dest, shape, ins, 1)) != XS_OK) return st;
@@ -477,6 +489,6 @@ const char *xs_get_error_string(xs_status status) {
 
 int xs_version(void) { return XS_VERSION; }
 
-const char *xs_last_error_detail(void) { return g_detail; }
+const char *xs_last_error_detail(void) { return xs::g_detail; }
 
 }  // extern "C"

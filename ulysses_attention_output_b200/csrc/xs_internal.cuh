@@ -139,4 +139,9 @@ cudaError_t launch_partial_empty(float *o, float *lse, long long rows, int D, cu
 
 int device_sm_count();
 
+// The detail string xs_last_error_detail() returns on this thread: record_error sets it
+// (printf-style) and returns `code`; clear_error empties it.
+int record_error(int code, const char *fmt, ...);
+void clear_error();
+
 }  // namespace xs
