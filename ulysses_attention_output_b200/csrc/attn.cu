@@ -28,8 +28,9 @@
 //   cols [384,512) O1
 // The MMA issue order per key tile j is QK0(j+1), PV1(j), QK1(j+1), PV0(j+1), so each tile's
 // softmax overlaps the other tile's two MMAs.  The running maximum is only moved when a new
-// row maximum exceeds it by more than 2^8 (in the exp2 domain); P then stays below 256 and
-// the rescale of O (done by the softmax thread itself, after the previous P V completed) is
+// row maximum exceeds it by more than 32 (in the exp2 domain); P then stays below 2^32, so O
+// and l stay below 2^32 * S * max|v| and 2^32 * S, far inside the fp32 range, and the rescale
+// of O (done by the softmax thread itself, after the previous P V completed) is
 // rare (the previous P V is complete by then: it precedes the Q K^T whose result the
 // softmax has just read).  P V consumes the probabilities rounded to bf16, and l sums those same rounded values
 // in fp32, so the normalised weights of every row add up to one.  The softmax works on column
@@ -45,7 +46,12 @@ constexpr int kThreads = 320;
 constexpr int kStages = 3;           // K/V ring slots
 constexpr int kStageRows = 16;       // rows staged per warp per epilogue round (head-major / partial)
 constexpr int kChunkBytes = 16384;   // 128 rows x 128 bytes (64 bf16) per swizzle panel
-constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest tolerated P before rescale
+// A rescale makes the whole warp reload and store O; with keys of outlying norm a threshold of
+// 8 made that happen in most key tiles of some warp (4% slower on such inputs than 32).
+#ifndef XS_RESCALE_LOG2
+#define XS_RESCALE_LOG2 32
+#endif
+constexpr float kRescaleThreshold = XS_RESCALE_LOG2;  // log2 of the largest tolerated P before rescale
 
 // TMEM column of S_t / P_t and of O_t for Q tile t.
 __host__ __device__ constexpr uint32_t col_s(int t) { return 128u * static_cast<uint32_t>(t); }
