@@ -401,12 +401,15 @@ def alloc_dest(B: int, H: int, S: int, D: int, P: int, device=None, fill: float 
 class HostPipeline:
     """End-to-end call with host buffers: pinned host q/k/v in, pinned host slabs out.
 
-    The heads are split into ``chunks`` groups that flow through three streams: host-to-device
+    The heads are split into ``chunks`` groups that flow through four streams: host-to-device
     copies of a group's q, k, v (input-copy stream), the fused per-rank call for that group's
-    heads writing every slab at the group's head offset (the caller's stream), and
-    device-to-host copies of those heads' columns of every slab (output-copy stream, one
-    2-D copy per slab).  The copies of one group overlap the kernels of the others; events
-    order each group's stages and, across calls, the reuse of its buffers.  ``run`` makes the
+    heads writing every slab at the group's head offset (the caller's stream for even groups,
+    a second compute stream for odd ones), and device-to-host copies of those heads' columns
+    of every slab (output-copy stream, one 2-D copy per slab).  The copies of one group
+    overlap the kernels of the others; with two compute streams the next group's kernel takes
+    each SM that the current one's last wave of work items leaves idle (one CTA of the kernel
+    fits an SM, so the two never share one).  Events order each group's stages and, across
+    calls, the reuse of its buffers.  ``run`` makes the
     caller's stream wait for every copy it started, so work timed on that stream covers the
     whole step.  ``chunks=1`` runs copies, kernel and copies in sequence on the caller's stream.
     Device buffers are allocated once, here, by PyTorch.
@@ -422,7 +425,8 @@ class HostPipeline:
         self.device = dev
         if chunks is None:
             # about one wave of 256-row work items per group, at most 20 groups (on the video
-            # workload 20 groups gave 24.2 ms per step, 8 gave 25.4, 4 gave 26.0, 1 gave 43.0)
+            # workload, with two compute streams: 20 groups 21.5-22.0 ms per step, 40 gave 21.6,
+            # 10 gave 22.7, 8 gave 23.0; one compute stream and 20 groups 24.2; 1 group 43.0)
             sms = torch.cuda.get_device_properties(dev).multi_processor_count
             items_per_head = B * ((S + 255) // 256)
             chunks = max(1, min(20, H, (H * items_per_head) // sms))
@@ -437,6 +441,7 @@ class HostPipeline:
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.s_in = torch.cuda.Stream(device=dev)
         self.s_out = torch.cuda.Stream(device=dev)
+        self.s_k2 = torch.cuda.Stream(device=dev)   # kernels of the odd groups
         n = len(self.groups)
         self.ev_in = [torch.cuda.Event() for _ in range(n)]     # group's inputs on the device
         self.ev_kern = [torch.cuda.Event() for _ in range(n)]   # group's kernel done
@@ -476,6 +481,7 @@ class HostPipeline:
         start.record(s)
         self.s_in.wait_event(start)
         self.s_out.wait_event(start)
+        self.s_k2.wait_event(start)
         for g, (h0, h1) in enumerate(self.groups):
             # inputs: the group's buffers are free once its previous kernel is done
             with torch.cuda.stream(self.s_in):
@@ -487,12 +493,13 @@ class HostPipeline:
                     self.v[g][b].copy_(v_host[b, h0:h1], non_blocking=True)
                 self.ev_in[g].record(self.s_in)
             # kernel: its inputs have landed and its slab columns have been copied out
-            s.wait_event(self.ev_in[g])
+            ks = s if g % 2 == 0 else self.s_k2
+            ks.wait_event(self.ev_in[g])
             if self._started:
-                s.wait_event(self.ev_out[g])
+                ks.wait_event(self.ev_out[g])
             attn_a2a_fused_rank(self.q[g], self.k[g], self.v[g], self.dest, heads_total=H,
-                                head_offset=h0, scale=self.scale, stream=s, status=self.status)
-            self.ev_kern[g].record(s)
+                                head_offset=h0, scale=self.scale, stream=ks, status=self.status)
+            self.ev_kern[g].record(ks)
             # outputs: the group's heads in every slab, one 2-D copy per slab
             self.s_out.wait_event(self.ev_kern[g])
             width = (h1 - h0) * D * 2
