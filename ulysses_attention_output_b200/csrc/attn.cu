@@ -34,7 +34,7 @@
 // rare (the previous P V is complete by then: it precedes the Q K^T whose result the
 // softmax has just read).  P V consumes the probabilities rounded to bf16, and l sums those same rounded values
 // in fp32, so the normalised weights of every row add up to one.  The softmax works on column
-// pairs in packed fp32 (f32x2) and computes 5 of every 16 pairs of exponentials with an FMA-pipe
+// pairs in packed fp32 (f32x2) and computes 4 of every 16 pairs of exponentials with an FMA-pipe
 // polynomial instead of MUFU ex2, because at one exponential per 4*D FLOPs MUFU alone would
 // take as long as the tensor core.
 #include "xs_internal.cuh"
@@ -81,7 +81,7 @@ __device__ __forceinline__ uint32_t f2u(float x) { return __float_as_uint(x); }
 // Column pairs (of 64 per 128-key tile) whose exponentials run on the FMA pipe instead of
 // MUFU: kEmulatedPer16 of every 16 pairs, spread evenly.
 #ifndef XS_EMULATED_PER16
-#define XS_EMULATED_PER16 5
+#define XS_EMULATED_PER16 4  // 3..7 measured: 4 fastest (2-3% ahead of 5, 3 and 6)
 #endif
 constexpr int kEmulatedPer16 = XS_EMULATED_PER16;
 __host__ __device__ constexpr bool emulated_pair(int c) {
