@@ -99,3 +99,18 @@ def gather_rows_from_slabs(dest, w_shape, rows: np.ndarray) -> np.ndarray:
 def workload_inputs(name):
     w = W.WORKLOADS[name]
     return w, W.make_inputs(w)
+
+
+def rising_scores(B, H, S, D, seed, steps=(0.0, 1.23, 4.7)):
+    """Q > 0 and key tile j offset by steps[j]: every row's maximum grows by 18-22 (exp2
+    domain, D = 64, S = 384) at the second key tile, below the lazy-rescale threshold of 32
+    (P up to ~2^22, no rescale), and the third tile's maximum lies 70-82 above the kept one,
+    which rescales O and l."""
+    g = torch.Generator().manual_seed(seed)
+    q = (1.0 + 0.5 * torch.randn((B, H, S, D), generator=g).abs()).to(torch.bfloat16)
+    k = 0.1 * torch.randn((B, H, S, D), generator=g)
+    for j, c in enumerate(steps):
+        k[:, :, 128 * j:128 * (j + 1)] += c
+    k = k.to(torch.bfloat16)
+    v = torch.randn((B, H, S, D), generator=g).to(torch.bfloat16)
+    return q, k, v

@@ -16,7 +16,7 @@ import oracle
 import ulysses_attention_output_b200 as xs
 from ulysses_attention_output_b200 import workloads as W
 
-from _parity import (assert_close, gather_rows_from_slabs, run_attn, run_fused, run_serial,
+from _parity import (assert_close, rising_scores, gather_rows_from_slabs, run_attn, run_fused, run_serial,
                      slabs_f64, to_gpu)
 
 pytestmark = pytest.mark.gpu
@@ -80,6 +80,32 @@ def test_attention_matches_oracle_every_row(B, H, S, D, P, structure):
     dest, st = run_fused(qg, kg, vg, P)
     assert st == 0
     assert_close(slabs_f64(dest), oracle.a2a_post(ref, P), f"fused {B,H,S,D,P}")
+
+
+def test_lazy_and_forced_rescale_paths():
+    """Rows whose maximum moves by less, then by more than the lazy-rescale threshold: the
+    fused and head-major outputs match the oracle (a skipped or misapplied rescale of O would
+    mix contributions of different scale)."""
+    B, H, S, D, P = 1, 4, 384, 64, 2
+    q, k, v = rising_scores(B, H, S, D, seed=21)
+    ref = oracle.attention(q, k, v)
+    qg, kg, vg = to_gpu(q, k, v)
+    out, st = run_attn(qg, kg, vg)
+    assert st == 0
+    assert_close(out.double().cpu().numpy(), ref, "rescale head-major")
+    dest, st = run_fused(qg, kg, vg, P)
+    assert st == 0
+    assert_close(slabs_f64(dest), oracle.a2a_post(ref, P), "rescale fused")
+
+
+def test_sixteen_ranks_fused():
+    """P = 16 (the largest rank count): 6-row slabs, work items straddling many slabs."""
+    B, H, S, D, P = 2, 16, 96, 128, 16
+    q, k, v = W.make_qkv(B, H, S, D, seed=1616)
+    ref = oracle.attention(q, k, v)
+    dest, st = run_fused(*to_gpu(q, k, v), P)
+    assert st == 0
+    assert_close(slabs_f64(dest), oracle.a2a_post(ref, P), "fused P=16")
 
 
 def test_explicit_scale():

@@ -22,7 +22,7 @@ import oracle
 import ulysses_attention_output_b200 as xs
 from ulysses_attention_output_b200 import workloads as W
 
-from _parity import assert_close, errors, run_attn
+from _parity import assert_close, errors, rising_scores, run_attn
 
 pytestmark = pytest.mark.gpu
 
@@ -71,6 +71,16 @@ def test_partial_matches_oracle(B, H, Sq, Skv, D, scale):
     ro, rl = oracle.attention_partial(q, k, v, scale=scale)
     assert_close(o, ro, f"partial O {B, H, Sq, Skv, D}")
     _check_lse(lse, rl, f"partial lse {B, H, Sq, Skv, D}")
+
+
+def test_partial_with_rescale_matches_oracle():
+    """Partial attention whose row maxima move below, then above the lazy-rescale threshold
+    (``rising_scores``): O and the lse match the oracle."""
+    q, k, v = rising_scores(1, 2, 384, 64, seed=33)
+    ref_o, ref_l = oracle.attention_partial(q, k, v)
+    o, lse = _partial_gpu(q, k, v)
+    assert_close(o, ref_o, "partial rescale O")
+    _check_lse(lse, ref_l, "partial rescale")
 
 
 def test_partial_empty_shard():
