@@ -426,7 +426,8 @@ class HostPipeline:
         if chunks is None:
             # about one wave of 256-row work items per group, at most 20 groups (on the video
             # workload, with two compute streams: 20 groups 21.5-22.0 ms per step, 40 gave 21.6,
-            # 10 gave 22.7, 8 gave 23.0; one compute stream and 20 groups 24.2; 1 group 43.0)
+            # 10 gave 22.7, 8 gave 23.0; one compute stream and 20 groups 24.2; 1 group 43.0;
+            # halving the first and last group, whose copies overlap no kernel, was 1-2% slower)
             sms = torch.cuda.get_device_properties(dev).multi_processor_count
             items_per_head = B * ((S + 255) // 256)
             chunks = max(1, min(20, H, (H * items_per_head) // sms))
