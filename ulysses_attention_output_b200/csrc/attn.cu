@@ -69,7 +69,8 @@ struct Smem {
   static constexpr uint32_t kRowPtr = kStage + kStageBytes;           // 8 x 16 pointers
   static constexpr uint32_t kBars = kRowPtr + 8 * kStageRows * 8;
   // barriers: q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_done[2] drain
-  static constexpr uint32_t kNumBars = 2 + 2 + kStages + kStages + 2 + 2 + 2 + 1;
+  //           p_lo[2]
+  static constexpr uint32_t kNumBars = 2 + 2 + kStages + kStages + 2 + 2 + 2 + 1 + 2;
   static constexpr uint32_t kMisc = kBars + kNumBars * 8;             // tmem base, abort flag
   static constexpr uint32_t kTotal = kMisc + 16;
   static constexpr size_t kAlloc = kTotal + 1024;                     // room for alignment
@@ -131,6 +132,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   auto p_full = [&](int t) { return bar0 + 8u * (6 + 2 * kStages + t); };
   auto o_done = [&](int t) { return bar0 + 8u * (8 + 2 * kStages + t); };
   const uint32_t drain_bar = bar0 + 8u * (10 + 2 * kStages);
+  // P of keys 0-63 of tile t stored (p_full: all of P): the MMA thread starts P V on that half
+  // while the softmax computes the other.
+  auto p_lo = [&](int t) { return bar0 + 8u * (11 + 2 * kStages + t); };
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(base + L::kMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(base + L::kMisc + 4);
 
@@ -143,6 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       ptx::mbar_init(q_empty(t), 1);
       ptx::mbar_init(s_full(t), 1);
       ptx::mbar_init(p_full(t), 4);  // one arrival per softmax warp
+      ptx::mbar_init(p_lo(t), 4);
       ptx::mbar_init(o_done(t), 1);
     }
     for (int s = 0; s < kStages; ++s) {
@@ -246,12 +251,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           ptx::mma_ss(d, a + off, b + off, idesc_qk, ks > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int t, uint32_t slot, bool acc) {
+      // P V over keys [64 half, 64 half + 64): four K steps of 16 keys.
+      auto issue_pv = [&](int t, uint32_t slot, bool acc, int half) {
         const uint64_t b = dv0 + static_cast<uint64_t>(slot) * kTileDesc;
         const uint32_t d = tmem + col_o(t);
         const uint32_t a = tmem + col_s(t);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
+        for (int ks = 4 * half; ks < 4 * half + 4; ++ks) {
           // A = P (bf16 pairs in TMEM, 8 columns per 16 keys); B = V tile, MN-major:
           // LBO = distance between 64-column panels, SBO = 8 key rows.
           ptx::mma_ts(d, a + ks * 8, b + static_cast<uint64_t>(ks * (2048 >> 4)), idesc_pv,
@@ -280,11 +286,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           ok = bounded_wait(kv_full(slotV), (kv_it / kStages) & 1u, ctl);
           if (!ok) break;
           ++kv_it;
+          ok = bounded_wait(p_lo(0), pc0 & 1u, ctl);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          issue_pv(0, slotV, j > 0, 0);
           ok = bounded_wait(p_full(0), pc0 & 1u, ctl);
           if (!ok) break;
           ++pc0;
           ptx::tc_fence_after();
-          issue_pv(0, slotV, j > 0);
+          issue_pv(0, slotV, true, 1);
           const bool more = (j + 1) < n_kv;
           // The s_full commit after QK_t(j+1) also covers PV_t(j), issued just before it, so
           // o_done is only needed for the last key tile (the epilogue waits for it).
@@ -299,11 +309,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             ptx::mma_commit(s_full(0));
             if (j + 2 == n_kv) ptx::mma_commit(q_empty(0));
           }
+          ok = bounded_wait(p_lo(1), pc1 & 1u, ctl);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          issue_pv(1, slotV, j > 0, 0);
           ok = bounded_wait(p_full(1), pc1 & 1u, ctl);
           if (!ok) break;
           ++pc1;
           ptx::tc_fence_after();
-          issue_pv(1, slotV, j > 0);
+          issue_pv(1, slotV, true, 1);
           if (!more) ptx::mma_commit(o_done(1));
           ptx::mma_commit(kv_empty(slotV));
           if (more) {
@@ -390,6 +404,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         // columns as P (the P words of chunk c land in columns [16c, 16c+16); the whole row
         // was read in pass 1).  (Re-reading S from TMEM here, chunk by chunk, was 1.5-2% slower.)
         // A fixed subset of the pairs uses the FMA-pipe exponential instead of MUFU.
+        // P is handed over in two halves (keys 0-63: p_lo, then all: p_full), so that P V on
+        // the first half runs while the second is computed.
         const uint64_t sl2x2 = ptx::f2x(sl2, sl2);
         const uint64_t negm2 = ptx::f2x(-m_run, -m_run);
         uint64_t lacc0 = 0, lacc1 = 0;  // packed row sums (0 bits == +0.0f)
@@ -425,6 +441,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         // The scores of pass 1 are still in registers: no second TMEM load.
         exp_chunk(0, reinterpret_cast<uint32_t(&)[32]>(sr[0]));
         exp_chunk(1, reinterpret_cast<uint32_t(&)[32]>(sr[32]));
+        if (__any_sync(0xffffffffu, rescale)) {
+          // O holds P V of the previous key tiles, all complete: PV_t(j-1) was issued before
+          // QK_t(j), whose completion (s_full) this thread has waited for.  Done before any P
+          // of this key tile is handed over (P V of its first half starts at p_lo), after the
+          // first half's exponentials, whose scores no longer need registers.
+          // 16 columns at a time: the second half's scores still occupy 64 registers.
+          const float a = rescale ? alpha : 1.f;
+#pragma unroll 1
+          for (int cc = 0; cc < DCH * 4; ++cc) {
+            uint32_t o[16];
+            ptx::tmem_ld16(tO + cc * 16, o);
+            ptx::tmem_wait_ld();
+            ptx::reg_fence16(o);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(u2f(o[i]) * a);
+            ptx::tmem_st16(tO + cc * 16, o);
+          }
+        }
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(p_lo(t));  // one arrival per warp
         exp_chunk(2, reinterpret_cast<uint32_t(&)[32]>(sr[64]));
         exp_chunk(3, reinterpret_cast<uint32_t(&)[32]>(sr[96]));
         {
@@ -432,21 +470,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           ptx::f2x_split(lacc0, a0, a1);
           ptx::f2x_split(lacc1, b0, b1);
           l_run += (a0 + a1) + (b0 + b1);
-        }
-        if (__any_sync(0xffffffffu, rescale)) {
-          // O holds P V of the previous key tiles, all complete: PV_t(j-1) was issued before
-          // QK_t(j), whose completion (s_full) this thread has waited for.
-          const float a = rescale ? alpha : 1.f;
-#pragma unroll
-          for (int cc = 0; cc < DCH * 2; ++cc) {
-            uint32_t o[32];
-            ptx::tmem_ld32(tO + cc * 32, o);
-            ptx::tmem_wait_ld();
-            ptx::reg_fence32(o);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(u2f(o[i]) * a);
-            ptx::tmem_st32(tO + cc * 32, o);
-          }
         }
         ptx::tmem_wait_st();
         ptx::tc_fence_before();

@@ -136,6 +136,14 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// The same for 16 values.
+__device__ __forceinline__ void reg_fence16(uint32_t *r) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
+                 "+r"(r[13]), "+r"(r[14]), "+r"(r[15]));
+}
+
 // Register fence: ties 32 values loaded by tcgen05.ld to a point after tcgen05.wait::ld, so
 // the compiler cannot move their first use above the wait.
 __device__ __forceinline__ void reg_fence32(uint32_t *r) {

@@ -8,6 +8,9 @@ measured dense bf16 peak; fused / serial and fused / attention-only; the exchang
 (2 B H S D 2 bytes) against the measured copy bandwidth.
 
 Run ``python -m ulysses_attention_output_b200.perf_table`` on a GPU; it prints one JSON object.
+``--vendor`` adds, as context only, the cuDNN attention kernel behind torch's
+``scaled_dot_product_attention`` (attention alone, no exchange, head-major output) on the same
+tensors, timed the same way.
 """
 from __future__ import annotations
 
@@ -26,7 +29,7 @@ def _peaks():
         return 1590.0, 1400.0, 6650.0, "fallback"
 
 
-def measure(name: str, reps: int = 21, warmup: int = 3) -> dict:
+def measure(name: str, reps: int = 21, warmup: int = 3, vendor: bool = False) -> dict:
     import torch
 
     import ulysses_attention_output_b200 as xs
@@ -45,6 +48,14 @@ def measure(name: str, reps: int = 21, warmup: int = 3) -> dict:
         "relayout": lambda: xs.a2a_relayout(out, dest),
         "serial": lambda: (xs.attn(q, k, v, out, status=status), xs.a2a_relayout(out, dest)),
     }
+    if vendor:
+        import torch.nn.functional as F
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+
+        def cudnn_sdpa():
+            with sdpa_kernel([SDPBackend.CUDNN_ATTENTION]):
+                F.scaled_dot_product_attention(q, k, v)
+        calls["vendor_cudnn"] = cudnn_sdpa
     samples = {key: [] for key in calls}
     for _ in range(warmup):
         for fn in calls.values():
@@ -64,7 +75,12 @@ def measure(name: str, reps: int = 21, warmup: int = 3) -> dict:
     med = {key: sorted(vals)[len(vals) // 2] for key, vals in samples.items()}
     peak, peak_sus, hbm, src = _peaks()
     tflops = w.flops / (med["fused"] * 1e-3) / 1e12
+    extra = {}
+    if vendor:
+        extra = {"vendor_cudnn_tflops": w.flops / (med["vendor_cudnn"] * 1e-3) / 1e12,
+                 "fused_vs_vendor_cudnn": med["fused"] / med["vendor_cudnn"]}
     return {
+        **extra,
         "workload": name, "B": w.B, "H": w.H, "S": w.S, "D": w.D, "P": w.P, "structure": w.structure,
         "reps": reps, "ms": med, "fused_tflops": tflops, "frac_bf16_peak": tflops / peak,
         "frac_bf16_sustained": tflops / peak_sus,
@@ -80,8 +96,9 @@ def main(argv=None):
     ap = argparse.ArgumentParser(description="Per-workload timing table (fused, serial, parts)")
     ap.add_argument("--workloads", default="tiny,ditxl,mmdit,long,video")
     ap.add_argument("--reps", type=int, default=21)
+    ap.add_argument("--vendor", action="store_true", help="also time cuDNN attention (context)")
     a = ap.parse_args(argv)
-    print(json.dumps([measure(n, a.reps) for n in a.workloads.split(",")]))
+    print(json.dumps([measure(n, a.reps, vendor=a.vendor) for n in a.workloads.split(",")]))
     return 0
 
 
