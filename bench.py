@@ -293,13 +293,16 @@ def oracle_sample(w, target_s: float):
 
 # ----------------------------------------------------------------------------- arms
 def workload_config(w, world: int = 1):
+    """The `config` object of both arms' lines (the same dict for the same workload and N)."""
     per_gpu = w.qkv_bytes // world
     return {"workload": w.name, "description": w.description, "B": w.B, "H": w.H, "S": w.S,
             "D": w.D, "P": w.P, "structure": w.structure,
             "l2": (f"inputs per GPU larger than L2 ({per_gpu / 2**20:.0f} MiB > 126 MiB), no flush"
                    if per_gpu > L2_BYTES else
                    f"inputs per GPU {per_gpu / 2**20:.0f} MiB fit in L2: a 252 MiB buffer is read "
-                   f"before every timed step, outside its events")}
+                   f"before every timed step, outside its events"),
+            "parallelism": (f"ulysses{world} (heads {w.H // world} per GPU, NVLink peer stores)"
+                            if world > 1 else "single")}
 
 
 def run_reference(args):
@@ -321,7 +324,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": workload_config(w),
+        "data": "synthetic", "config": workload_config(w, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": smp.threads, "kind": "oracle",
                          "sample": smp.describe(n, total / args.steps)},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -500,8 +503,6 @@ def run_xs(args):
         "scaling": "strong" if world > 1 else "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {**workload_config(w, world),
-                   "parallelism": f"ulysses{world} (heads {w.H // world} per GPU, NVLink peer stores)"
-                   if world > 1 else "single",
                    **({"dist_backend": "gloo (host-ordered check, not a measurement)"}
                       if world > 1 and args.dist_backend == "gloo" else {})},
         "frac_of_bf16_peak": achieved / peak,
@@ -511,6 +512,11 @@ def run_xs(args):
         "relayout_gbs": relayout_gbs, "relayout_frac_hbm": relayout_gbs / hbm,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
+                     "traffic_source": (f"dram__bytes_read.sum + dram__bytes_write.sum per launch from the "
+                                        f"committed ncu summary profiles/attn_fused_{w.name}.md, taken on "
+                                        f"kernel sources of the same digest ({source_digest()}); not "
+                                        f"measured in this run" if traffic is not None else
+                                        "no ncu capture of these kernel sources"),
                      "peak_source": f"{peak_src} bf16 burst", "peak_sustained": peak_sus,
                      "frac_sustained": achieved / peak_sus, "kernel": "attn_fwd_kernel<2,kSeqScatter>"},
         "e2e": e2e, "cpu_baseline": cpu, "clocks": clk.summary(),

@@ -97,6 +97,45 @@ XS_API xs_status xs_attn_a2a_fused_rank(const void *q, const void *k, const void
                                         int *dev_status);
 
 /*
+ * xs_attn_a2a_fused_rank that also publishes, per destination slab, an arrival counter: the
+ * device-initiated completion signal of the one-sided stores (X-Stage abstract: the exchange
+ * is made of device-initiated one-sided remote stores; explainer "FlashAttention-A2A
+ * (Piggybacking)": the tile's owner stores it into the destination rank's shard).  Arguments
+ * and results as xs_attn_a2a_fused_rank, plus:
+ *   slab_flags : HOST array of shape.P device pointers; slab_flags[r] is one 32-bit counter,
+ *                4-byte aligned, that lives with slab r (on the GPU that owns it, which may be
+ *                another GPU reachable by peer access), outside every slab and input.  Distinct.
+ * After storing its rows of a tile, each storing warp adds the number of rows it stored into
+ * slab r to *slab_flags[r] with a system-scope release, so a reader that observes the counter
+ * with an acquire load also observes those rows.  One complete call adds
+ * B * (S / P) * shape.H to every slab's counter.  Counters only grow (mod 2^32): a caller
+ * that reuses them across steps waits for the running total (see xs_slab_wait) instead of
+ * clearing them, or clears them (cudaMemsetAsync) in stream order before the call.
+ * The storing warps wait for their own stores to become visible before each release; this
+ * is done by the warps that store, after they have handed the tile's accumulator back, so
+ * the attention's key loop does not wait for it.
+ */
+XS_API xs_status xs_attn_a2a_fused_flags(const void *q, const void *k, const void *v,
+                                         void *const *dest, unsigned int *const *slab_flags,
+                                         xs_shape shape, int heads_total, int head_offset,
+                                         float scale, xs_stream_t stream, int *dev_status);
+
+/*
+ * Consumer side of the arrival counters: enqueue on `stream` a wait until *flag has reached
+ * `target` (compared modulo 2^32: the wait ends once flag - target, as a signed 32-bit
+ * value, is >= 0).  One GPU thread polls the counter with system-scope acquire loads; work
+ * enqueued on `stream` after this call sees every row that the counted releases covered.
+ *   flag       : device pointer (this GPU's memory or a peer's), 4-byte aligned.
+ *   limit_ns   : 1e3 <= limit_ns <= 1e11; after that much global time the wait gives up and
+ *                writes XS_ERR_TIMEOUT to *dev_status (device int, required).
+ * On one GPU the wait must be ordered after the producing call (same stream, or an event):
+ * a waiting kernel and the kernel it waits for are not guaranteed to run at the same time on
+ * one device.  Across GPUs the producers run on their own devices.
+ */
+XS_API xs_status xs_slab_wait(const unsigned int *flag, unsigned int target, long long limit_ns,
+                              xs_stream_t stream, int *dev_status);
+
+/*
  * xs_attn_a2a_fused with a record of the sender-visible store-issue span of every output
  * tile (the quantity the X-Stage explainer's Burst-Gap model describes: "Methodik: Die
  * X-Stage-Abstraktion und das Burst-Gap-Modell").  Same arguments and results as
@@ -229,8 +268,11 @@ XS_API xs_status xs_burst_probe(void *scratch, long long scratch_bytes, xs_burst
  *     HBM-drain measurements use xs_burst_probe with a buffer larger than L2.
  *   - burst_bytes above XS_BURST_STATIC_SCRATCH_BYTES is rejected with XS_ERR_UNSUPPORTED;
  *     other limits and the stamps layout are those of xs_burst_probe.
- *   - The first call on a device looks up the array's device address (once per device, with
- *     that device current); make that first call before any stream capture.
+ *   - Every call looks up the array's device address in the CUDA context current on the
+ *     calling thread (cudaGetSymbolAddress, which allocates nothing), so callers that switch
+ *     contexts or reset the device get the right address.  The first call in a context may
+ *     load the library's device code into it: make that first call before any stream
+ *     capture.
  *   - No cudaMalloc, cudaFree or allocating library routine is called.
  *   - Every call shares the one array and leaves its contents behind; the probe only stores
  *     into it, so nothing needs to start at zero.  Calls that overlap on the GPU (other
@@ -248,6 +290,24 @@ XS_API xs_status xs_burst_probe_static(xs_burst_cfg cfg, unsigned long long *sta
  * to *dev_status (device, required).  The context stays usable afterwards.
  */
 XS_API xs_status xs_selftest_bounded_wait(int *dev_status, long long limit_ns, xs_stream_t stream);
+
+/*
+ * Self-test of the attention kernel's own abort path.  Runs xs_attn (head-major output) with
+ * two changes: every CTA's TMA producer stops before its fill number `stall_fill` (Q and K/V
+ * tile fills of that CTA counted together from 0), as if that copy never arrived, and every
+ * on-device wait gives up after limit_ns nanoseconds of global time instead of the
+ * library's 2 s.  The waits that depend on the missing fill then run out: the kernel writes
+ * XS_ERR_TIMEOUT to *dev_status, each CTA lets the copies and MMAs it already started
+ * finish, frees its tensor memory and returns, and the context stays usable.  `out` is left
+ * partly written.  Arguments as xs_attn, plus:
+ *   stall_fill : >= 0; a CTA that needs fewer fills completes normally.
+ *   limit_ns   : 1e3 <= limit_ns <= 1e10.
+ *   dev_status : device int, required.
+ * A test entry point: no page of the method describes it.
+ */
+XS_API xs_status xs_selftest_attn_abort(const void *q, const void *k, const void *v, void *out,
+                                        xs_shape shape, int stall_fill, long long limit_ns,
+                                        xs_stream_t stream, int *dev_status);
 
 /*
  * Peer mapping of destination slabs between the processes of one node (one process per

@@ -80,6 +80,31 @@ def test_fused_rejects_pointers(lib):
     assert "overlaps" in detail
 
 
+def test_flags_and_wait_reject(lib):
+    shape = xs.Shape(1, 4, 256, 64, 2)
+    q, k, v = FAKE, FAKE + 30 * MB, FAKE + 60 * MB
+    dest = (ctypes.c_void_p * 2)(FAKE + 100 * MB, FAKE + 200 * MB)
+
+    def call(flags, sh=shape, ht=4, off=0):
+        arr = (ctypes.c_void_p * 2)(*flags) if flags is not None else None
+        return lib.xs_attn_a2a_fused_flags(q, k, v, dest, arr, sh, ht, off, 0.0, None, None)
+
+    assert call(None) == xs.XS_ERR_INVALID_ARG                                        # no array
+    assert call([FAKE + 300 * MB, 0]) == xs.XS_ERR_INVALID_ARG                        # null counter
+    assert call([FAKE + 300 * MB, FAKE + 300 * MB + 2]) == xs.XS_ERR_INVALID_ARG      # misaligned
+    assert call([FAKE + 300 * MB, FAKE + 300 * MB]) == xs.XS_ERR_INVALID_ARG          # same counter
+    assert call([FAKE + 300 * MB, FAKE + 100 * MB + 64]) == xs.XS_ERR_INVALID_ARG     # inside a slab
+    assert "inside dest" in lib.xs_last_error_detail().decode()
+    assert call([FAKE + 300 * MB, FAKE + 64]) == xs.XS_ERR_INVALID_ARG                # inside q
+    assert call([FAKE + 300 * MB, FAKE + 301 * MB], off=2) == xs.XS_ERR_INVALID_ARG   # heads past the layer
+    assert call([FAKE + 300 * MB, FAKE + 301 * MB], sh=xs.Shape(1, 4, 256, 60, 2)) == xs.XS_ERR_UNSUPPORTED
+    st = FAKE + 400 * MB
+    assert lib.xs_slab_wait(0, 1, 10 ** 6, None, st) == xs.XS_ERR_INVALID_ARG
+    assert lib.xs_slab_wait(FAKE + 2, 1, 10 ** 6, None, st) == xs.XS_ERR_INVALID_ARG
+    assert lib.xs_slab_wait(FAKE, 1, 10 ** 6, None, 0) == xs.XS_ERR_INVALID_ARG
+    assert lib.xs_slab_wait(FAKE, 1, 10, None, st) == xs.XS_ERR_INVALID_ARG
+
+
 def test_attn_and_relayout_reject(lib):
     sh = xs.Shape(1, 4, 256, 64, 2)
     assert lib.xs_attn(FAKE, FAKE + MB, FAKE + 2 * MB, 0, sh, 0.0, None, None) == xs.XS_ERR_INVALID_ARG
@@ -98,6 +123,15 @@ def test_probe_and_selftest_reject(lib):
     assert lib.xs_burst_probe(FAKE, 1 << 20, xs.BurstCfg(4096, 4, 0, 8, 100), FAKE + 8 * MB, None) == xs.XS_ERR_INVALID_ARG
     assert lib.xs_selftest_bounded_wait(0, 10 ** 6, None) == xs.XS_ERR_INVALID_ARG
     assert lib.xs_selftest_bounded_wait(FAKE, 10, None) == xs.XS_ERR_INVALID_ARG
+    sh = xs.Shape(1, 2, 256, 64, 1)
+    q, k, v, out = FAKE, FAKE + MB, FAKE + 2 * MB, FAKE + 3 * MB
+    # every bad argument is refused on the host, before anything is enqueued
+    assert lib.xs_selftest_attn_abort(q, k, v, out, sh, 0, 10 ** 6, None, 0) == xs.XS_ERR_INVALID_ARG
+    assert lib.xs_selftest_attn_abort(q, k, v, out, sh, -1, 10 ** 6, None, FAKE + 4 * MB) == xs.XS_ERR_INVALID_ARG
+    assert lib.xs_selftest_attn_abort(q, k, v, out, sh, 0, 10, None, FAKE + 4 * MB) == xs.XS_ERR_INVALID_ARG
+    assert lib.xs_selftest_attn_abort(q, k, v, q, sh, 0, 10 ** 6, None, FAKE + 4 * MB) == xs.XS_ERR_INVALID_ARG
+    assert lib.xs_selftest_attn_abort(q, k, v, out, xs.Shape(1, 2, 256, 60, 1), 0, 10 ** 6, None,
+                                      FAKE + 4 * MB) == xs.XS_ERR_UNSUPPORTED
 
 
 def test_binding_has_no_fallback(monkeypatch, tmp_path):

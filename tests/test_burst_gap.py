@@ -93,3 +93,82 @@ def test_span_stats_from_synthetic_stamps():
     assert sum(r["hist_counts"]) == 12
     # an explicit clock rate overrides the estimate
     assert abs(bg.span_stats(st, grid, ghz=1.0)["span_ns"]["p50"] - 2450.0) < 1e-6
+
+
+# ----------------------------------------------------------------------------- knee and capacity
+def knee_points(v, t0, r, gaps, noise=0.0, seed=0, slope=1.0):
+    """Points of one (K, V) over G from the model (slope != 1 plants a model violation)."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for g in gaps:
+        t = max(t0, v / r - slope * g) * (1 + noise * rng.standard_normal())
+        out.append({"K": 148, "V": v, "G_ns": float(g), "t_iss_ns": t})
+    return out
+
+
+def test_fit_knee_recovers_t0_r_and_knee():
+    v, t0, r = 64 << 20, 7600.0, 7700.0                  # bytes, ns, bytes/ns (= GB/s)
+    gaps = np.linspace(0.0, 2 * v / r, 17)
+    f = bg.fit_knee(knee_points(v, t0, r, gaps))
+    assert abs(f["R_GBps"] - r) / r < 1e-6
+    assert abs(f["T0_ns"] - t0) < 1e-6
+    assert abs(f["knee_G_ns"] - (v / r - t0)) < 1e-3
+    assert abs(f["free_slope"] - 1.0) < 1e-6
+    assert f["rms_rel_residual"] < 1e-9
+
+
+def test_fit_knee_with_noise_and_a_planted_slope():
+    v, t0, r = 128 << 20, 15000.0, 7000.0
+    gaps = np.linspace(0.0, 2 * v / r, 33)
+    f = bg.fit_knee(knee_points(v, t0, r, gaps, noise=0.01, seed=4))
+    assert abs(f["R_GBps"] - r) / r < 0.03
+    assert abs(f["free_slope"] - 1.0) < 0.15
+    # a drain side of slope 0.5 instead of 1 is not the model: the free slope shows it
+    g = bg.fit_knee(knee_points(v, t0, r, gaps, slope=0.5))
+    assert abs(g["free_slope"] - 0.5) < 0.05
+
+
+def test_fit_knee_without_a_drain_regime():
+    """Every gap beyond the knee (backpressure-free only): no drain-side points, no R."""
+    v, t0 = 8 << 20, 1000.0
+    f = bg.fit_knee(knee_points(v, t0, 1e9, np.linspace(0.0, 5000.0, 9)))
+    assert f["drain_points"] == 0 and f["R_GBps"] is None and abs(f["T0_ns"] - t0) < 1e-9
+
+
+def test_knee_report_predicts_a_held_out_volume():
+    r, c, issue = 7500.0, 200.0, 8800.0
+    mib = 1 << 20
+    pts = []
+    for v in (32 * mib, 64 * mib, 96 * mib, 128 * mib):
+        pts += knee_points(v, c + v / issue, r, np.linspace(0.0, 2 * v / r, 17))
+    rep = bg.knee_report(pts, 96 * mib)
+    assert abs(rep["R_GBps_mean"] - r) / r < 1e-6
+    assert rep["prediction_rms_rel"] < 1e-9
+    assert rep["prediction_drain_side_points"] > 0
+    # a held-out curve that breaks the model is predicted badly
+    bad = [p if p["V"] != 96 * mib else {**p, "t_iss_ns": 1.3 * p["t_iss_ns"]} for p in pts]
+    assert bg.knee_report(bad, 96 * mib)["prediction_rms_rel"] > 0.2
+
+
+def capacity_points(vols, c, issue, q, drain):
+    return [{"K": 148, "V": v, "G_ns": 1e6, "t_iss_ns": c + min(v, q) / issue + max(v - q, 0) / drain}
+            for v in vols]
+
+
+def test_fit_capacity_recovers_q():
+    mib = 1 << 20
+    vols = [v * mib for v in (8, 16, 32, 48, 64, 96, 128, 192, 256, 384, 512)]
+    f = bg.fit_capacity(capacity_points(vols, 250.0, 8800.0, 96 * mib, 6000.0))
+    assert f["Q_bytes"] == 96 * mib
+    assert abs(f["issue_GBps"] - 8800.0) / 8800.0 < 1e-6
+    assert abs(f["drain_GBps"] - 6000.0) / 6000.0 < 1e-6
+    assert f["rms_rel_residual"] < 1e-9 < f["one_line_rms_rel_residual"]
+
+
+def test_fit_capacity_without_a_break():
+    """One rate over every volume: Q is beyond the largest burst measured."""
+    mib = 1 << 20
+    vols = [v * mib for v in (8, 16, 32, 64, 128, 256)]
+    f = bg.fit_capacity(capacity_points(vols, 250.0, 8000.0, 1 << 40, 8000.0))
+    assert f["Q_bytes"] is None or abs(f["issue_GBps"] - f["drain_GBps"]) / 8000.0 < 1e-6
+    assert abs(f["one_line_GBps"] - 8000.0) / 8000.0 < 1e-6

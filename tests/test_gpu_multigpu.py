@@ -4,8 +4,10 @@ process stores its finished tiles into both processes' slabs.  The processes are
 the host (stream synchronisation + a gloo barrier), so no kernel waits on another.
 
 Checked bit for bit against the single-process fused call on all heads (itself checked
-against the oracle by the parity tests): the fused multi-process step, and the serial step
-(attention, pack, all-to-all, unpack).  Every slab is filled with NaN bits first, so a
+against the oracle by the parity tests): the fused multi-process step, the serial step
+(attention, pack, all-to-all, unpack), and the fused step with arrival counters (each
+process's warps release-add their row counts to the owning process's counters through the
+IPC mapping; the counts must come out exact).  Every slab is filled with NaN bits first, so a
 missing store fails the comparison.
 """
 import os
@@ -80,9 +82,22 @@ def _steps(case, dev):
     layer.serial(ql, kl, vl, out, send, recv, status=status)
     layer.complete()
     serial_ok = matches()
+    layer.complete()
+
+    # arrival counters: each process's stores add to the owner's counters (IPC-mapped); the
+    # host orders both processes' fused calls before either waits, so the waits find their
+    # counts already there and no kernel spins while another on this GPU produces
+    layer.slabs.view(torch.int16).fill_(-1)
+    layer.complete()
+    layer.fused_flags(ql, kl, vl, status=status)
+    layer.complete()
+    target = layer.wait_slabs(status=status)
+    flags_ok = matches() and target == layer.rows_per_slab and \
+        [int(c) for c in layer.counters.cpu()] == [layer.rows_per_slab] * pl.slabs_local
     st = int(status.item())
+    layer.complete()
     layer.close()
-    return fused_ok, serial_ok, st, len(layer.dest)
+    return fused_ok, serial_ok and flags_ok, st, len(layer.dest)
 
 
 @pytest.mark.parametrize("case", CASES)
@@ -106,4 +121,5 @@ def test_two_process_fused_exchange_bit_exact(case, cuda_device):
         assert st == 0, f"device status {st} on process {rank}"
         assert n_dest == case[4]
         assert fused_ok, f"fused multi-process slabs of process {rank} differ from the single fused call"
-        assert serial_ok, f"serial multi-process slabs of process {rank} differ from the single fused call"
+        assert serial_ok, (f"serial (or flagged) multi-process slabs or arrival counts of process {rank} "
+                           "differ from the single fused call")

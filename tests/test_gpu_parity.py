@@ -3,8 +3,9 @@
 * the exchange pass moves every 16-bit word to the oracle's slot (bit-exact, sentinels and
   canaries checked);
 * attention (head-major) and fused attention + exchange match the fp64 oracle within
-  max-abs 2e-2 and rel-L2 5e-3 -- every row for small and ragged shapes, sampled rows
-  (always including sequence ends and rank boundaries) for the long workloads;
+  max-abs 2e-2 and rel-L2 5e-3 -- every row for small and ragged shapes and for the tiny,
+  DiT-XL/2 and MMDiT workloads, sampled rows (always including sequence ends and rank
+  boundaries) for the long and video workloads;
 * the fused result equals attention followed by the separate exchange bit for bit, at every
   element of every workload (same kernel arithmetic, different store addresses).
 """
@@ -132,7 +133,7 @@ def test_constant_values_and_zero_queries():
     assert_close(out.double().cpu().numpy(), mean, "Q = 0")
 
 
-@pytest.mark.parametrize("name", ["tiny", "ditxl"])
+@pytest.mark.parametrize("name", ["tiny", "ditxl", "mmdit"])
 def test_workload_every_row(name):
     w = W.WORKLOADS[name]
     q, k, v = W.make_inputs(w)
@@ -147,7 +148,7 @@ def test_workload_every_row(name):
         assert torch.equal(a.view(torch.int16), b.view(torch.int16)), "fused != attention + exchange"
 
 
-@pytest.mark.parametrize("name,n_rows", [("mmdit", 512), ("long", 256), ("video", 256)])
+@pytest.mark.parametrize("name,n_rows", [("long", 256), ("video", 256)])
 def test_workload_sampled_rows(name, n_rows):
     w = W.WORKLOADS[name]
     q, k, v = W.make_inputs(w)

@@ -91,6 +91,15 @@ def _layer_worker(rank, world, port, out_q):
             base = layer.slabs.data_ptr() if g == rank else FAKE_BASE * (g + 1) + FAKE_OFFSET
             expect.append(base + i * nb)
         table_ok = layer.dest == expect
+        # arrival counters: right after each GPU's P/N slabs, 256 bytes apart
+        cexp = []
+        for r in range(P):
+            g, i = divmod(r, pl.slabs_local)
+            base = layer.slabs.data_ptr() if g == rank else FAKE_BASE * (g + 1) + FAKE_OFFSET
+            cexp.append(base + pl.slabs_local * nb + 256 * i)
+        table_ok = table_ok and layer.flag_table == cexp and \
+            layer.counters.data_ptr() == layer.slabs.data_ptr() + pl.slabs_local * nb and \
+            int(layer.counters.abs().sum()) == 0 and layer.rows_per_slab == B * (S // P) * H
 
         # serial exchange: pack this GPU's heads per rank, all-to-all, unpack
         rng = np.random.default_rng(11)

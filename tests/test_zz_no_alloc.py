@@ -7,7 +7,11 @@ a fixed 32 MiB array inside the library.  Both entry points run the same kernel,
 the same configuration and a scratch ring of the same size their stamps must agree: every
 (producer, burst) record written and ordered, the compute-gap cycles within 10 % (a fixed
 dependent FMA chain) and the median issue cycles within a factor of 3 (store issue timing
-varies run to run).  Checked on two calls in a row.  This file is collected last.
+varies run to run).  Checked on two calls in a row.  The property the entry point exists
+for is checked as well: across calls after the first, neither torch's allocator counters nor
+the device's free memory (cudaMemGetInfo) move.  A burst of exactly the array's size, the
+largest accepted and the edge of the cyclic walk, writes every stamp.  This file is
+collected last.
 """
 import ctypes
 
@@ -75,3 +79,35 @@ def test_static_probe_rejects_oversize_burst(lib):
     assert b"exceeds the fixed" in lib.xs_last_error_detail()
     torch.cuda.synchronize()
     assert (stamps == 0).all()  # nothing was launched
+
+
+def test_static_probe_allocates_nothing(lib):
+    """After a first call (which may load the library's device code), further calls change
+    neither torch's allocation counters nor the device's free memory."""
+    stamps = torch.zeros((PRODUCERS, N_BURSTS, 4), dtype=torch.int64, device="cuda")
+    cfg = xs.BurstCfg(BURST, PRODUCERS, GAP, N_BURSTS, THREADS)
+    assert lib.xs_burst_probe_static(cfg, stamps.data_ptr(), None) == xs.XS_OK
+    torch.cuda.synchronize()
+    stats0 = torch.cuda.memory_stats()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        assert lib.xs_burst_probe_static(cfg, stamps.data_ptr(), None) == xs.XS_OK
+    torch.cuda.synchronize()
+    stats1 = torch.cuda.memory_stats()
+    free1, _ = torch.cuda.mem_get_info()
+    for key in ("allocation.all.allocated", "segment.all.allocated", "reserved_bytes.all.current"):
+        assert stats1.get(key, 0) == stats0.get(key, 0), key
+    assert free1 == free0
+
+
+def test_static_probe_burst_of_the_whole_array(lib):
+    """burst_bytes == XS_BURST_STATIC_SCRATCH_BYTES: every producer's share fills its part of
+    the array exactly once per burst; all records are written and ordered."""
+    n = 3
+    stamps = torch.zeros((PRODUCERS, n, 4), dtype=torch.int64, device="cuda")
+    cfg = xs.BurstCfg(STATIC_BYTES, PRODUCERS, 0, n, THREADS)
+    rc = lib.xs_burst_probe_static(cfg, stamps.data_ptr(), None)
+    assert rc == xs.XS_OK, lib.xs_last_error_detail()
+    torch.cuda.synchronize()
+    st = stamps.cpu()
+    assert (st[..., 0] > 0).all() and (st[..., 1] >= st[..., 0]).all() and (st[..., 2] >= st[..., 1]).all()

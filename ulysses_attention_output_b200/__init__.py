@@ -11,12 +11,15 @@ Calls (same names as the C ABI, without the ``xs_`` prefix):
 * :func:`a2a_relayout`   -- the exchange as a separate pass (serial baseline).
 * :func:`attn_a2a_fused_rank` -- the fused call of one Ulysses rank (its heads, all slabs).
 * :func:`attn_a2a_fused_spans` -- the fused call, also recording each tile's store-issue span.
+* :func:`attn_a2a_fused_flags` -- the fused call, also publishing per-slab arrival counters.
+* :func:`slab_wait`      -- bounded wait of a consumer until a slab's counter reaches a target.
 * :func:`a2a_pre`        -- the pre-attention exchange (sequence shards -> head-major).
 * :func:`attn_partial`   -- partial attention over one key/value shard, fp32 output + lse.
 * :func:`lse_merge`      -- online-softmax merge of partial results (the Route primitive).
 * :func:`burst_probe`    -- Burst-Gap store microbenchmark.
 * :func:`burst_probe_static` -- the same, with no device allocation (fixed library scratch).
 * :func:`selftest_bounded_wait` -- exercises the bounded on-device wait.
+* :func:`selftest_attn_abort` -- makes the attention kernel's own waits run out (abort path).
 """
 from __future__ import annotations
 
@@ -28,7 +31,8 @@ __all__ = [
     "XsError", "XS_OK", "XS_ERR_INVALID_ARG", "XS_ERR_UNSUPPORTED", "XS_ERR_CUDA", "XS_ERR_TIMEOUT",
     "library_path", "load", "version", "attn_a2a_fused", "attn", "a2a_relayout", "burst_probe",
     "attn_a2a_fused_rank", "a2a_pre", "attn_partial", "lse_merge", "attn_a2a_fused_spans",
-    "burst_probe_static", "selftest_bounded_wait", "alloc_dest", "HostPipeline", "attention_flops",
+    "burst_probe_static", "selftest_bounded_wait", "selftest_attn_abort", "alloc_dest",
+    "attn_a2a_fused_flags", "slab_wait", "HostPipeline", "attention_flops",
     "ipc_export", "ipc_open", "ipc_close", "IPC_HANDLE_BYTES",
 ]
 
@@ -90,6 +94,9 @@ def load():
         lib.xs_burst_probe.argtypes = [vp, ctypes.c_longlong, BurstCfg, vp, vp]
         lib.xs_burst_probe_static.argtypes = [BurstCfg, vp, vp]
         lib.xs_selftest_bounded_wait.argtypes = [ip, ctypes.c_longlong, vp]
+        lib.xs_selftest_attn_abort.argtypes = [vp, vp, vp, vp, Shape, c_int, ctypes.c_longlong, vp, ip]
+        lib.xs_attn_a2a_fused_flags.argtypes = [vp, vp, vp, vpp, vpp, Shape, c_int, c_int, c_float, vp, ip]
+        lib.xs_slab_wait.argtypes = [vp, ctypes.c_uint, ctypes.c_longlong, vp, ip]
         lib.xs_attn_partial.argtypes = [vp, vp, vp, vp, vp, Shape, c_int, c_float, vp, ip]
         lib.xs_attn_a2a_fused_spans.argtypes = [vp, vp, vp, vpp, Shape, c_float, vp, ctypes.c_longlong, vp, ip]
         lib.xs_lse_merge.argtypes = [vpp, vpp, c_int, vp, vp, ctypes.c_longlong, c_int, vp]
@@ -97,7 +104,8 @@ def load():
         lib.xs_ipc_open.argtypes = [ctypes.c_char_p, ctypes.POINTER(ctypes.c_void_p)]
         lib.xs_ipc_close.argtypes = [vp]
         for fn in (lib.xs_attn_a2a_fused, lib.xs_attn, lib.xs_a2a_relayout, lib.xs_burst_probe,
-                   lib.xs_burst_probe_static, lib.xs_selftest_bounded_wait,
+                   lib.xs_burst_probe_static, lib.xs_selftest_bounded_wait, lib.xs_selftest_attn_abort,
+                   lib.xs_attn_a2a_fused_flags, lib.xs_slab_wait,
                    lib.xs_attn_a2a_fused_rank, lib.xs_a2a_pre, lib.xs_attn_partial, lib.xs_lse_merge,
                    lib.xs_attn_a2a_fused_spans):
             fn.restype = c_int
@@ -222,6 +230,52 @@ def attn_a2a_fused_rank(q, k, v, dest, heads_total: int, head_offset: int, scale
     _check(load().xs_attn_a2a_fused_rank(q.data_ptr(), k.data_ptr(), v.data_ptr(), arr, shp,
                                          int(heads_total), int(head_offset), float(scale or 0.0),
                                          _stream_handle(stream), _ptr(status)))
+
+
+def attn_a2a_fused_flags(q, k, v, dest, flags, heads_total: int | None = None, head_offset: int = 0,
+                         scale: float | None = None, stream=None, status=None):
+    """:func:`attn_a2a_fused_rank` that also adds, after storing, each slab's row count to its
+    arrival counter ``flags[r]`` (an int32/uint32 CUDA tensor element, or an int address of a
+    counter mapped from another process) with a system-scope release.  ``heads_total``
+    defaults to this call's own head count (the single-GPU fused call)."""
+    P = len(dest)
+    if len(flags) != P:
+        raise ValueError(f"{len(flags)} counters for {P} slabs")
+    shp = _shape_of(q, P)
+    ht = shp.H if heads_total is None else int(heads_total)
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _bf16_cuda(n, t, tuple(q.shape))
+    ptrs = []
+    for r, d in enumerate(dest):
+        if isinstance(d, int):
+            ptrs.append(d)
+        else:
+            _bf16_cuda(f"dest[{r}]", d, (shp.B, shp.S // P, ht, shp.D))
+            ptrs.append(d.data_ptr())
+    fptrs = [f if isinstance(f, int) else _counter_ptr(f"flags[{r}]", f) for r, f in enumerate(flags)]
+    arr = (ctypes.c_void_p * P)(*ptrs)
+    farr = (ctypes.c_void_p * P)(*fptrs)
+    _check(load().xs_attn_a2a_fused_flags(q.data_ptr(), k.data_ptr(), v.data_ptr(), arr, farr, shp,
+                                          ht, int(head_offset), float(scale or 0.0),
+                                          _stream_handle(stream), _ptr(status)))
+
+
+def _counter_ptr(name: str, t) -> int:
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype not in (torch.int32, torch.uint32):
+        raise TypeError(f"{name} must be a 32-bit integer CUDA tensor (one element)")
+    if t.numel() < 1:
+        raise ValueError(f"{name} is empty")
+    return t.data_ptr()
+
+
+def slab_wait(flag, target: int, limit_ns: int, status, stream=None):
+    """Enqueue a wait until the arrival counter ``flag`` reaches ``target`` (modulo 2^32);
+    after ``limit_ns`` it gives up and ``status`` (int32 CUDA tensor) receives XS_ERR_TIMEOUT.
+    On one GPU, order it after the producing call (stream or event)."""
+    fp = flag if isinstance(flag, int) else _counter_ptr("flag", flag)
+    _check(load().xs_slab_wait(fp, int(target) & 0xFFFFFFFF, int(limit_ns), _stream_handle(stream),
+                               status.data_ptr()))
 
 
 def ipc_export(t) -> tuple[bytes, int]:
@@ -382,6 +436,18 @@ def burst_probe_static(stamps, burst_bytes: int, producers: int, gap_cycles: int
 def selftest_bounded_wait(status, limit_ns: int, stream=None):
     """Launch the bounded-wait self-test; ``status`` (int32 CUDA tensor) receives XS_ERR_TIMEOUT."""
     _check(load().xs_selftest_bounded_wait(status.data_ptr(), int(limit_ns), _stream_handle(stream)))
+
+
+def selftest_attn_abort(q, k, v, out, status, stall_fill: int, limit_ns: int, stream=None):
+    """Head-major attention whose TMA producer stops before fill ``stall_fill`` of every CTA and
+    whose waits give up after ``limit_ns``: ``status`` (int32 CUDA tensor, required) receives
+    XS_ERR_TIMEOUT and the kernel returns; ``out`` is left partly written."""
+    shp = _shape_of(q, 1)
+    for n, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+        _bf16_cuda(n, t, tuple(q.shape))
+    _check(load().xs_selftest_attn_abort(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                         shp, int(stall_fill), int(limit_ns),
+                                         _stream_handle(stream), status.data_ptr()))
 
 
 def alloc_dest(B: int, H: int, S: int, D: int, P: int, device=None, fill: float | None = None):

@@ -26,7 +26,10 @@ ring in this GPU's memory, i.e. the local stand-in for remote stores) over a gri
 issuer waits until its stores have drained (issue time V / R for every burst, no overlap).
 
 Run ``python -m ulysses_attention_output_b200.burst_gap [--large] [--wide] [--fused] [--spans]``
-on a GPU for a sweep (``--large``: bursts of 4..64 MB from 148 producers; ``--wide``: 1024
+or ``--knee`` on a GPU for a sweep (``--large``: bursts of 4..64 MB from 148 producers;
+``--knee``: G swept densely through the knee at 32..128 MiB with one volume held out and
+predicted from the others' fit, plus drained single bursts up to 512 MiB for the outstanding
+capacity Q; ``--wide``: 1024
 threads per producer; ``--fused``: also time the fused kernel against attention alone on the
 MMDiT, long and video workloads and set the measured overhead beside both models'
 predictions; ``--spans``: the per-tile store-issue span histogram of the fused kernel,
@@ -277,6 +280,140 @@ def store_spans(points, names=("mmdit", "long", "video")):
     return out
 
 
+# ----------------------------------------------------------------------------- knee and capacity
+def fit_knee(points):
+    """Fit T_iss(G) = max(T0_iss, V/R - G) for the points of ONE (K, V), swept over G.
+
+    The drain-dominated side has slope -1 in G by the model; the fit splits the points at
+    every candidate knee, takes T0_iss as the mean issue time beyond it and V/R as the mean of
+    t + G before it, and keeps the split with the least squared error.  Also fitted, as a
+    check of the model rather than a parameter of it: the free slope b of t = a - b G over
+    the drain-side points (the model says b = 1).  Returns T0_ns, R_GBps (bytes per ns), the
+    knee G* = V/R - T0_iss, the free slope, the number of drain-side points and the RMS
+    relative residual of the fitted max(.) curve over all points."""
+    pts = sorted(points, key=lambda p: p["G_ns"])
+    v = float(pts[0]["V"])
+    g = np.array([p["G_ns"] for p in pts], dtype=np.float64)
+    t = np.array([p["t_iss_ns"] for p in pts], dtype=np.float64)
+    best = None
+    for split in range(0, len(pts) + 1):  # points [0, split) drain side, [split, n) floor
+        if split == len(pts):
+            continue  # no floor point: T0 undetermined
+        t0 = float(t[split:].mean())
+        a = float((t[:split] + g[:split]).mean()) if split else t0  # a = V / R
+        model = np.maximum(t0, a - g)
+        sse = float(((model - t) ** 2).sum())
+        if best is None or sse < best[0]:
+            best = (sse, split, t0, a)
+    _, split, t0, a = best
+    model = np.maximum(t0, a - g)
+    rms = float(np.sqrt(np.mean(((model - t) / t) ** 2)))
+    slope = None
+    if split >= 2:
+        b, _ = np.polyfit(g[:split], t[:split], 1)
+        slope = float(-b)
+    r = v / a if split else None
+    return {"K": pts[0]["K"], "V": int(v), "T0_ns": t0, "R_GBps": r,
+            "knee_G_ns": (a - t0) if split else None, "drain_points": int(split),
+            "free_slope": slope, "rms_rel_residual": rms}
+
+
+def fit_capacity(points):
+    """Outstanding capacity Q from single bursts with a gap long enough for every earlier
+    burst to have drained (points of one K over V, G beyond V/R).  Below Q the burst is
+    absorbed at the issue rate I; beyond it issue stalls and the rest goes at the drain rate:
+    t(V) = c + V / I for V <= Q, t(V) = c + Q / I + (V - Q) / R_q above.  Q is scanned over
+    the measured volumes (and left as "beyond the largest" when one line fits best).
+    Returns c, I, R_q, Q and the RMS relative residual."""
+    pts = sorted(points, key=lambda p: p["V"])
+    v = np.array([p["V"] for p in pts], dtype=np.float64)
+    t = np.array([p["t_iss_ns"] for p in pts], dtype=np.float64)
+    best = None
+    for qi in range(1, len(pts)):  # Q = v[qi]: points 0..qi on the first line
+        q = v[qi]
+        # least squares in (c, 1/I, 1/R): t = c + min(V, Q)/I + max(V - Q, 0)/R
+        a = np.stack([np.ones_like(v), np.minimum(v, q), np.maximum(v - q, 0.0)], axis=1)
+        coef, *_ = np.linalg.lstsq(a, t, rcond=None)
+        sse = float(((a @ coef - t) ** 2).sum())
+        if best is None or sse < best[0] - 1e-12 * sse:
+            best = (sse, q, coef)
+    _, q, coef = best
+    c, inv_i, inv_r = (float(x) for x in coef)
+    model = c + np.minimum(v, q) * inv_i + np.maximum(v - q, 0.0) * inv_r
+    one = np.polyfit(v, t, 1)
+    one_rms = float(np.sqrt(np.mean(((np.polyval(one, v) - t) / t) ** 2)))
+    rms = float(np.sqrt(np.mean(((model - t) / t) ** 2)))
+    broken = q < v[-1] and inv_r > 0 and inv_i > 0
+    return {"c_ns": c, "issue_GBps": 1.0 / inv_i if inv_i > 0 else None,
+            "drain_GBps": 1.0 / inv_r if inv_r > 0 else None, "Q_bytes": int(q) if broken else None,
+            "rms_rel_residual": rms, "one_line_rms_rel_residual": one_rms,
+            "one_line_GBps": 1.0 / one[0] if one[0] > 0 else None}
+
+
+def knee_sweep(volumes, k: int = 148, r_guess_gbs: float = 7700.0, ghz_guess: float = 1.9,
+               n_gaps: int = 17, n_bursts: int = 48, drop: int = 8, threads: int = 256,
+               scratch_bytes: int = 2 << 30):
+    """T_iss over G densely through [0, 2 V/R] (R guessed) for each V at K producers."""
+    import torch
+
+    import ulysses_attention_output_b200 as xs
+    scratch = torch.empty(scratch_bytes, dtype=torch.uint8, device="cuda")
+    out = []
+    for v in volumes:
+        vv = (v // (16 * k)) * 16 * k
+        g_max_cycles = 2.0 * vv / r_guess_gbs * ghz_guess
+        for i in range(n_gaps):
+            g = int(round(g_max_cycles * i / (n_gaps - 1)))
+            out.append(run_point(xs, torch, scratch, k, vv, g, n_bursts, threads, drop))
+    del scratch
+    return out
+
+
+def capacity_sweep(volumes, k: int = 148, r_guess_gbs: float = 5000.0, ghz_guess: float = 1.9,
+                   n_bursts: int = 12, drop: int = 4, threads: int = 256,
+                   scratch_bytes: int = 2 << 30):
+    """Single bursts separated by a gap of 3 V/R (R guessed low): every burst starts drained."""
+    import torch
+
+    import ulysses_attention_output_b200 as xs
+    scratch = torch.empty(scratch_bytes, dtype=torch.uint8, device="cuda")
+    out = []
+    for v in volumes:
+        vv = (v // (16 * k)) * 16 * k
+        g = int(3.0 * vv / r_guess_gbs * ghz_guess)
+        out.append(run_point(xs, torch, scratch, k, vv, g, n_bursts, threads, drop))
+    del scratch
+    return out
+
+
+def knee_report(points, held_out_v: int):
+    """Per-V knee fits of the volumes other than held_out_v, R from their mean, T0_iss(V)
+    from a line through their floors, and the prediction of the held-out volume's whole
+    T_iss(G) curve against its measurement (relative error per point and RMS)."""
+    by_v = {}
+    for p in points:
+        by_v.setdefault(p["V"], []).append(p)
+    fits = {v: fit_knee(pts) for v, pts in sorted(by_v.items())}
+    train = [f for v, f in fits.items() if v != held_out_v and f["R_GBps"]]
+    r = float(np.mean([f["R_GBps"] for f in train]))
+    vols = np.array([f["V"] for f in train], dtype=np.float64)
+    floors = np.array([f["T0_ns"] for f in train], dtype=np.float64)
+    line = np.polyfit(vols, floors, 1) if len(train) >= 2 else (0.0, floors[0])
+    t0_pred = float(np.polyval(line, held_out_v))
+    check = []
+    for p in sorted(by_v.get(held_out_v, []), key=lambda q: q["G_ns"]):
+        pred = predict(t0_pred, r, held_out_v, p["G_ns"])
+        check.append({"G_ns": p["G_ns"], "measured_ns": p["t_iss_ns"], "predicted_ns": pred,
+                      "rel_err": (pred - p["t_iss_ns"]) / p["t_iss_ns"]})
+    rms = float(np.sqrt(np.mean([c["rel_err"] ** 2 for c in check]))) if check else None
+    drain_side = [c for c in check if held_out_v / r - c["G_ns"] > t0_pred]
+    return {"fits": list(fits.values()), "R_GBps_mean": r,
+            "R_GBps_spread": float(np.ptp([f["R_GBps"] for f in train])) if train else None,
+            "held_out_V": held_out_v, "T0_pred_ns": t0_pred, "knee_pred_G_ns": held_out_v / r - t0_pred,
+            "prediction": check, "prediction_rms_rel": rms,
+            "prediction_drain_side_points": len(drain_side)}
+
+
 def main(argv=None):
     argv = sys.argv[1:] if argv is None else argv
     volumes = [4096 << i for i in range(11)]         # 4 KB .. 4 MB
@@ -286,6 +423,18 @@ def main(argv=None):
         volumes = [4 << 20, 8 << 20, 16 << 20, 32 << 20, 64 << 20]
         producers = [148]
     threads = 1024 if "--wide" in argv else 256
+    if "--knee" in argv:
+        # G swept through the knee V/R - T0_iss at 148 producers; 96 MiB is held out of the
+        # fit and predicted; then single drained bursts up to 512 MiB for the capacity Q.
+        mib = 1 << 20
+        kp = knee_sweep([32 * mib, 64 * mib, 96 * mib, 128 * mib], threads=threads)
+        held = (96 * mib // (16 * 148)) * 16 * 148
+        cp = capacity_sweep([v * mib for v in (8, 16, 32, 48, 64, 96, 128, 192, 256, 384, 512)],
+                            threads=threads)
+        print(json.dumps({"threads_per_producer": threads, "knee_points": kp,
+                          "knee": knee_report(kp, held), "capacity_points": cp,
+                          "capacity": fit_capacity(cp)}))
+        return 0
     pts = sweep(volumes, producers, gaps, threads=threads)
     res = {"threads_per_producer": threads, "points": pts, "fit": fit(pts)}
     if "--fused" in argv:

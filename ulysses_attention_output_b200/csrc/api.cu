@@ -3,6 +3,7 @@
 // synchronises: every call only enqueues work on the caller's stream.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -153,6 +154,7 @@ xs_status fill_attention(xs::AttnParams &p, const void *q, const void *k, const 
   p.scale_log2 = static_cast<float>(sc * 1.4426950408889634);  // scale * log2(e)
   p.status = dev_status;
   p.wait_limit_ns = xs::kWaitLimitNs;
+  p.stall_fill = -1;  // never (the self-test entry point alone sets it)
   return XS_OK;
 }
 
@@ -165,15 +167,16 @@ xs_status launched(cudaError_t e, const char *what) {
 
 namespace xs {
 int device_sm_count() {
-  static int cache[64] = {};
+  // Per-device cache; threads that race on a first call both store the same count.
+  static std::atomic<int> cache[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
-  if (cache[dev] == 0) {
-    int n = 0;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
-    cache[dev] = n;
+    cache[dev].store(n, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return n;
 }
 }  // namespace xs
 
@@ -253,6 +256,68 @@ xs_status xs_attn_a2a_fused_rank(const void *q, const void *k, const void *v, vo
   for (int r = 0; r < shape.P; ++r) p.dest[r] = dest[r];
   return launched(xs::launch_attention(p, xs::kSeqScatter, reinterpret_cast<cudaStream_t>(stream)),
                   "attention launch");
+}
+
+xs_status xs_attn_a2a_fused_flags(const void *q, const void *k, const void *v, void *const *dest,
+                                  unsigned int *const *slab_flags, xs_shape shape, int heads_total,
+                                  int head_offset, float scale, xs_stream_t stream,
+                                  int *dev_status) {
+  if (!slab_flags) return fail(XS_ERR_INVALID_ARG, "slab_flags must be a host array of P device pointers");
+  for (int r = 0; r < shape.P && r < XS_MAX_RANKS; ++r) {
+    if (!slab_flags[r] || (reinterpret_cast<uintptr_t>(slab_flags[r]) & 3u))
+      return fail(XS_ERR_INVALID_ARG, "slab_flags[%d] must be a 4-byte aligned device pointer", r);
+    for (int o = 0; o < r; ++o)
+      if (slab_flags[o] == slab_flags[r])
+        return fail(XS_ERR_INVALID_ARG, "slab_flags[%d] and slab_flags[%d] are the same counter", o, r);
+  }
+  xs_shape layer = shape;
+  layer.H = heads_total;
+  xs_status st = check_shape(layer, true);
+  if (st != XS_OK) return st;
+  if ((st = check_shape(shape, false)) != XS_OK) return st;
+  if (head_offset < 0 || shape.H > heads_total || head_offset > heads_total - shape.H)
+    return fail(XS_ERR_INVALID_ARG, "heads [%d, %d) are not inside the layer's %d heads", head_offset,
+                head_offset + shape.H, heads_total);
+  if ((st = check_inputs(q, k, v, shape)) != XS_OK) return st;
+  const void *ins[3] = {q, k, v};
+  if ((st = check_dest(dest, shape, ins, 3, heads_total)) != XS_OK) return st;
+  {
+    // a counter inside a slab or an input would be overwritten by the data it counts
+    const uintptr_t slab = static_cast<uintptr_t>(shape.B) * (shape.S / shape.P) * heads_total * shape.D * 2;
+    const uintptr_t full = static_cast<uintptr_t>(shape.B) * shape.H * shape.S * shape.D * 2;
+    for (int r = 0; r < shape.P; ++r) {
+      const Range f{reinterpret_cast<uintptr_t>(slab_flags[r]), reinterpret_cast<uintptr_t>(slab_flags[r]) + 4};
+      for (int o = 0; o < shape.P; ++o) {
+        const Range d{reinterpret_cast<uintptr_t>(dest[o]), reinterpret_cast<uintptr_t>(dest[o]) + slab};
+        if (overlap(f, d)) return fail(XS_ERR_INVALID_ARG, "slab_flags[%d] lies inside dest[%d]", r, o);
+      }
+      for (const void *in : {q, k, v}) {
+        const Range i{reinterpret_cast<uintptr_t>(in), reinterpret_cast<uintptr_t>(in) + full};
+        if (overlap(f, i)) return fail(XS_ERR_INVALID_ARG, "slab_flags[%d] lies inside an input", r);
+      }
+    }
+  }
+  xs::AttnParams p;
+  if ((st = fill_attention(p, q, k, v, shape, scale, dev_status)) != XS_OK) return st;
+  p.H_dest = heads_total;
+  p.head_offset = head_offset;
+  for (int r = 0; r < shape.P; ++r) {
+    p.dest[r] = dest[r];
+    p.slab_flags[r] = slab_flags[r];
+  }
+  return launched(xs::launch_attention(p, xs::kSeqScatter, reinterpret_cast<cudaStream_t>(stream)),
+                  "attention launch");
+}
+
+xs_status xs_slab_wait(const unsigned int *flag, unsigned int target, long long limit_ns,
+                       xs_stream_t stream, int *dev_status) {
+  if (!flag || (reinterpret_cast<uintptr_t>(flag) & 3u))
+    return fail(XS_ERR_INVALID_ARG, "flag must be a 4-byte aligned device pointer");
+  if (!dev_status) return fail(XS_ERR_INVALID_ARG, "dev_status is required");
+  if (limit_ns < 1000 || limit_ns > 100000000000LL)
+    return fail(XS_ERR_INVALID_ARG, "limit_ns out of range [1e3, 1e11]");
+  return launched(xs::launch_slab_wait(flag, target, limit_ns, dev_status, reinterpret_cast<cudaStream_t>(stream)),
+                  "slab wait launch");
 }
 
 xs_status xs_attn(const void *q, const void *k, const void *v, void *out, xs_shape shape,
@@ -474,6 +539,34 @@ xs_status xs_selftest_bounded_wait(int *dev_status, long long limit_ns, xs_strea
     return fail(XS_ERR_INVALID_ARG, "limit_ns out of range [1e3, 1e10]");
   return launched(xs::launch_wait_selftest(dev_status, limit_ns, reinterpret_cast<cudaStream_t>(stream)),
                   "self-test launch");
+}
+
+xs_status xs_selftest_attn_abort(const void *q, const void *k, const void *v, void *out,
+                                 xs_shape shape, int stall_fill, long long limit_ns,
+                                 xs_stream_t stream, int *dev_status) {
+  if (!dev_status) return fail(XS_ERR_INVALID_ARG, "dev_status is required");
+  if (stall_fill < 0) return fail(XS_ERR_INVALID_ARG, "stall_fill must be >= 0 (got %d)", stall_fill);
+  if (limit_ns < 1000 || limit_ns > 10000000000LL)
+    return fail(XS_ERR_INVALID_ARG, "limit_ns out of range [1e3, 1e10]");
+  xs_status st = check_shape(shape, false);
+  if (st != XS_OK) return st;
+  if ((st = check_inputs(q, k, v, shape)) != XS_OK) return st;
+  if (!out || !aligned16(out)) return fail(XS_ERR_INVALID_ARG, "out must be a 16-byte aligned device pointer");
+  {
+    const uintptr_t full = static_cast<uintptr_t>(shape.B) * shape.H * shape.S * shape.D * 2;
+    const Range o{reinterpret_cast<uintptr_t>(out), reinterpret_cast<uintptr_t>(out) + full};
+    for (const void *in : {q, k, v}) {
+      const Range r{reinterpret_cast<uintptr_t>(in), reinterpret_cast<uintptr_t>(in) + full};
+      if (overlap(o, r)) return fail(XS_ERR_INVALID_ARG, "out overlaps an input tensor");
+    }
+  }
+  xs::AttnParams p;
+  if ((st = fill_attention(p, q, k, v, shape, 0.f, dev_status)) != XS_OK) return st;
+  p.out = out;
+  p.wait_limit_ns = limit_ns;
+  p.stall_fill = stall_fill;
+  return launched(xs::launch_attention(p, xs::kHeadMajor, reinterpret_cast<cudaStream_t>(stream)),
+                  "attention self-test launch");
 }
 
 const char *xs_get_error_string(xs_status status) {

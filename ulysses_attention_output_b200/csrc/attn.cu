@@ -20,7 +20,8 @@
 //   warps 0-3  softmax for Q tile 0 (one thread per query row = one TMEM lane)
 //   warps 4-7  softmax for Q tile 1
 //   warp  8    TMA producer: Q tiles once per work item, then K_j, V_j through a 3-slot ring
-//   warp  9    TMEM allocator and single-thread tcgen05.mma issuer
+//   warp  9    TMEM allocator and tcgen05.mma issuer (the warp runs the loop, one elected
+//              lane issues)
 // A work item is 256 query rows (two 128-row tiles) of one (b, h).  Tensor memory holds
 //   cols [0,128)   S0 = Q0 K^T (fp32), overwritten in place by P0 (bf16 pairs, 64 cols)
 //   cols [128,256) S1 / P1
@@ -37,6 +38,8 @@
 // pairs in packed fp32 (f32x2) and computes 4 of every 16 pairs of exponentials with an FMA-pipe
 // polynomial instead of MUFU ex2, because at one exponential per 4*D FLOPs MUFU alone would
 // take as long as the tensor core.
+#include <mutex>
+
 #include "xs_internal.cuh"
 
 namespace xs {
@@ -108,8 +111,21 @@ __device__ __forceinline__ void exp2_fma_pair(uint64_t x2, float &p0, float &p1)
   float q0, q1, t0, t1;
   ptx::f2x_split(q, q0, q1);
   ptx::f2x_split(t, t0, t1);
-  p0 = u2f(f2u(q0) + (f2u(t0) << 23));
-  p1 = u2f(f2u(q1) + (f2u(t1) << 23));
+  // The low bits of t hold n (t = 1.5 * 2^23 + n exactly); n * 2^23 added to the bits of 2^f
+  // moves its exponent by n: one integer multiply-add per element.
+  p0 = u2f(ptx::mad_lo_u32(f2u(t0), 1u << 23, f2u(q0)));
+  p1 = u2f(ptx::mad_lo_u32(f2u(t1), 1u << 23, f2u(q1)));
+}
+
+// acc += the two bf16 halves of pk, each converted exactly and added with one fp32 rounding
+// (sm_100 mixed-precision add): two instructions per pair, no unpacking.
+__device__ __forceinline__ void madd2(uint64_t &acc, uint32_t pk) {
+  float a0, a1;
+  ptx::f2x_split(acc, a0, a1);
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+      : "+f"(a0), "+f"(a1) : "r"(pk));
+  acc = ptx::f2x(a0, a1);
 }
 
 template <int DCH, int EPI>
@@ -180,12 +196,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     if (lane == 0) {
       uint32_t kv_it = 0, it = 0;
       int q_filled0 = -1, q_filled1 = -1;
+      int fills = 0;  // Q and K/V tile fills started (self-test stall point)
       bool ok = true;
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++it) {
         const int bh = item / p.n_pairs;
         const int q0 = (item - bh * p.n_pairs) * 256;
         for (int t = 0; t < 2 && ok; ++t) {
-          ok = bounded_wait(q_empty(t), (it & 1u) ^ 1u, ctl);
+          ok = bounded_wait(q_empty(t), (it & 1u) ^ 1u, ctl) && fills++ != p.stall_fill;
           if (!ok) break;
           ptx::mbar_arrive_expect_tx(q_full(t), L::kTile);
           for (int c = 0; c < DCH; ++c)
@@ -197,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         for (int j = 0; j < n_kv && ok; ++j) {
           for (int kv = 0; kv < 2; ++kv) {
             const uint32_t slot = kv_it % kStages;
-            ok = bounded_wait(kv_empty(slot), ((kv_it / kStages) & 1u) ^ 1u, ctl);
+            ok = bounded_wait(kv_empty(slot), ((kv_it / kStages) & 1u) ^ 1u, ctl) && fills++ != p.stall_fill;
             if (!ok) break;
             ptx::mbar_arrive_expect_tx(kv_full(slot), L::kTile);
             const CUtensorMap *tm = kv == 0 ? &p.tm_k : &p.tm_v;
@@ -212,16 +229,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         // Abort: let every copy this thread started land before the CTA can exit.
         // The ring slots hold the last (up to) kStages fills, numbered kv_it - kStages .. kv_it - 1.
         for (uint32_t f = kv_it > kStages ? kv_it - kStages : 0; f < kv_it; ++f)
-          bounded_wait_drain(kv_full(f % kStages), (f / kStages) & 1u, p.wait_limit_ns);
+          bounded_wait_drain(kv_full(f % kStages), (f / kStages) & 1u, kDrainLimitNs);
         if (q_filled0 >= 0)
-          bounded_wait_drain(q_full(0), static_cast<uint32_t>(q_filled0) & 1u, p.wait_limit_ns);
+          bounded_wait_drain(q_full(0), static_cast<uint32_t>(q_filled0) & 1u, kDrainLimitNs);
         if (q_filled1 >= 0)
-          bounded_wait_drain(q_full(1), static_cast<uint32_t>(q_filled1) & 1u, p.wait_limit_ns);
+          bounded_wait_drain(q_full(1), static_cast<uint32_t>(q_filled1) & 1u, kDrainLimitNs);
       }
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the issue loop (waits, loop control, descriptor arithmetic, all
+    // warp-uniform) and one elected lane issues each MMA and commit.  Run by lane 0 alone,
+    // the same loop left the tensor core idle between MMA groups for long enough to cost
+    // up to 15% in a layout with more warps per SM.
+    {
       const int ks_d = (p.D + 15) >> 4;              // K steps of 16 covering the true D
       const uint32_t n_pv = static_cast<uint32_t>(ks_d * 16);   // N of P V (D padded to 16)
       const uint32_t idesc_qk = ptx::idesc_bf16_f32(128, 128, 0);
@@ -248,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 #pragma unroll
         for (int ks = 0; ks < DCH * 4; ++ks) {
           const uint64_t off = static_cast<uint64_t>(((ks >> 2) * kChunkBytes + (ks & 3) * 32) >> 4);
-          ptx::mma_ss(d, a + off, b + off, idesc_qk, ks > 0 ? 1u : 0u);
+          ptx::mma_ss_elect(d, a + off, b + off, idesc_qk, ks > 0 ? 1u : 0u);
         }
       };
       // P V over keys [64 half, 64 half + 64): four K steps of 16 keys.
@@ -260,37 +281,42 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         for (int ks = 4 * half; ks < 4 * half + 4; ++ks) {
           // A = P (bf16 pairs in TMEM, 8 columns per 16 keys); B = V tile, MN-major:
           // LBO = distance between 64-column panels, SBO = 8 key rows.
-          ptx::mma_ts(d, a + ks * 8, b + static_cast<uint64_t>(ks * (2048 >> 4)), idesc_pv,
+          ptx::mma_ts_elect(d, a + ks * 8, b + static_cast<uint64_t>(ks * (2048 >> 4)), idesc_pv,
                       (acc || ks > 0) ? 1u : 0u);
         }
       };
 
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++it) {
         ok = bounded_wait(q_full(0), it & 1u, ctl) && bounded_wait(q_full(1), it & 1u, ctl);
+        ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         uint32_t slotK = kv_it % kStages;
         ok = bounded_wait(kv_full(slotK), (kv_it / kStages) & 1u, ctl);
+        ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         ++kv_it;
         ptx::tc_fence_after();
         issue_qk(0, slotK);
-        ptx::mma_commit(s_full(0));
-        if (n_kv == 1) ptx::mma_commit(q_empty(0));
+        ptx::mma_commit_elect(s_full(0));
+        if (n_kv == 1) ptx::mma_commit_elect(q_empty(0));
         issue_qk(1, slotK);
-        ptx::mma_commit(s_full(1));
-        ptx::mma_commit(kv_empty(slotK));
-        if (n_kv == 1) ptx::mma_commit(q_empty(1));
+        ptx::mma_commit_elect(s_full(1));
+        ptx::mma_commit_elect(kv_empty(slotK));
+        if (n_kv == 1) ptx::mma_commit_elect(q_empty(1));
 
         for (int j = 0; j < n_kv && ok; ++j) {
           const uint32_t slotV = kv_it % kStages;
           ok = bounded_wait(kv_full(slotV), (kv_it / kStages) & 1u, ctl);
+          ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           ++kv_it;
           ok = bounded_wait(p_lo(0), pc0 & 1u, ctl);
+          ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           ptx::tc_fence_after();
           issue_pv(0, slotV, j > 0, 0);
           ok = bounded_wait(p_full(0), pc0 & 1u, ctl);
+          ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           ++pc0;
           ptx::tc_fence_after();
@@ -298,39 +324,42 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           const bool more = (j + 1) < n_kv;
           // The s_full commit after QK_t(j+1) also covers PV_t(j), issued just before it, so
           // o_done is only needed for the last key tile (the epilogue waits for it).
-          if (!more) ptx::mma_commit(o_done(0));
+          if (!more) ptx::mma_commit_elect(o_done(0));
           if (more) {
             slotK = kv_it % kStages;
             ok = bounded_wait(kv_full(slotK), (kv_it / kStages) & 1u, ctl);
+            ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             ++kv_it;
             // (no tcgen05 fence here: K arrived through TMA, no tensor-memory hand-off)
             issue_qk(0, slotK);
-            ptx::mma_commit(s_full(0));
-            if (j + 2 == n_kv) ptx::mma_commit(q_empty(0));
+            ptx::mma_commit_elect(s_full(0));
+            if (j + 2 == n_kv) ptx::mma_commit_elect(q_empty(0));
           }
           ok = bounded_wait(p_lo(1), pc1 & 1u, ctl);
+          ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           ptx::tc_fence_after();
           issue_pv(1, slotV, j > 0, 0);
           ok = bounded_wait(p_full(1), pc1 & 1u, ctl);
+          ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           ++pc1;
           ptx::tc_fence_after();
           issue_pv(1, slotV, true, 1);
-          if (!more) ptx::mma_commit(o_done(1));
-          ptx::mma_commit(kv_empty(slotV));
+          if (!more) ptx::mma_commit_elect(o_done(1));
+          ptx::mma_commit_elect(kv_empty(slotV));
           if (more) {
             issue_qk(1, slotK);
-            ptx::mma_commit(s_full(1));
-            ptx::mma_commit(kv_empty(slotK));
-            if (j + 2 == n_kv) ptx::mma_commit(q_empty(1));
+            ptx::mma_commit_elect(s_full(1));
+            ptx::mma_commit_elect(kv_empty(slotK));
+            if (j + 2 == n_kv) ptx::mma_commit_elect(q_empty(1));
           }
         }
       }
-      // Every MMA this thread issued must be complete before TMEM is released.
-      ptx::mma_commit(drain_bar);
-      bounded_wait_drain(drain_bar, 0, p.wait_limit_ns);
+      // Every MMA the elected lane issued must be complete before TMEM is released.
+      ptx::mma_commit_elect(drain_bar);
+      bounded_wait_drain(drain_bar, 0, kDrainLimitNs);
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
@@ -430,11 +459,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             }
             pk[c] = ptx::pack_bf16(p0, p1);
             // Row sum of the bf16-rounded probabilities, i.e. of exactly the weights P V uses.
-            const uint64_t r2 = ptx::f2x(u2f(pk[c] << 16), u2f(pk[c] & 0xffff0000u));
             if (c & 1)
-              lacc1 = ptx::add2(lacc1, r2);
+              madd2(lacc1, pk[c]);
             else
-              lacc0 = ptx::add2(lacc0, r2);
+              madd2(lacc0, pk[c]);
           }
           ptx::tmem_st16(tS + 16 * ch, pk);
         };
@@ -548,6 +576,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             }
           }
         }
+        if (p.slab_flags[0] != nullptr) {
+          // Arrival counters: after the warp's stores (ordered before the leader's release by
+          // the warp barrier), one lane per destination slab among the warp's 32 rows adds
+          // that slab's row count with a system-scope release.  The release waits for the
+          // warp's stores to become visible, so this path costs the storing warps that wait;
+          // without counters the stores are never waited for.
+          const int r = dst_row != nullptr ? s_row / p.S_local : -1;
+          __syncwarp();
+          unsigned pending = __ballot_sync(0xffffffffu, r >= 0);
+          while (pending != 0u) {
+            const int leader = __ffs(pending) - 1;
+            const int rl = __shfl_sync(0xffffffffu, r, leader);
+            const unsigned same = __ballot_sync(0xffffffffu, r == rl);
+            if (lane == leader) ptx::red_release_sys_add(p.slab_flags[rl], __popc(same));
+            pending &= ~same;
+          }
+        }
       } else {
         // Head-major and partial epilogues: rounds of kRows rows per warp (16 in bf16, 8 in
         // fp32) staged in shared memory (chunk order rotated by row to spread banks), then
@@ -635,22 +680,24 @@ template <int DCH, int EPI>
 cudaError_t launch_impl(const AttnParams &p, cudaStream_t stream) {
   using L = Smem<DCH>;
   static_assert(L::kAlloc <= 232448, "shared memory budget exceeded");
-  auto kern = attn_fwd_kernel<DCH, EPI>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  static bool configured[64] = {};
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(L::kAlloc));
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
+  constexpr int kMaxDevices = 64;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  // Per device, once (threads racing on a first call wait for the one that sets it up): the
+  // opt-in to the dynamic shared memory this instance needs.
+  static std::once_flag once[kMaxDevices];
+  static cudaError_t setup[kMaxDevices];
+  std::call_once(once[dev], [dev] {
+    setup[dev] = cudaFuncSetAttribute(attn_fwd_kernel<DCH, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(L::kAlloc));
+  });
+  if (setup[dev] != cudaSuccess) return setup[dev];
   const int sms = device_sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
   const int grid = p.n_items < sms ? p.n_items : sms;
-  kern<<<grid, kThreads, L::kAlloc, stream>>>(p);
+  attn_fwd_kernel<DCH, EPI><<<grid, kThreads, L::kAlloc, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -1,7 +1,5 @@
 // exchange.cu -- the stand-alone post-attention All-to-All (serial baseline), the Burst-Gap
 // store microbenchmark and the bounded-wait self-test.
-#include <mutex>
-
 #include "xs_internal.cuh"
 
 namespace xs {
@@ -149,31 +147,47 @@ __global__ void wait_selftest_kernel(int *status, long long limit_ns) {
   }
 }
 
+// ---------------------------------------------------------------- slab arrival wait
+// One thread polls the counter with system-scope acquire loads, sleeping between polls, until
+// it reaches target or the limit passes (then XS_ERR_TIMEOUT is recorded).  Stream order makes
+// the kernels enqueued after this one see every store the counted releases covered.
+__global__ void slab_wait_kernel(const unsigned int *flag, unsigned int target, long long limit_ns,
+                                 int *status) {
+  const uint64_t t0 = ptx::globaltimer();
+  while (static_cast<int>(ptx::ld_acquire_sys(flag) - target) < 0) {
+    if (static_cast<long long>(ptx::globaltimer() - t0) > limit_ns) {
+      atomicCAS(status, kStatusOk, kStatusTimeout);
+      return;
+    }
+    __nanosleep(1000);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_slab_wait(const unsigned int *flag, unsigned int target, long long limit_ns,
+                             int *status, cudaStream_t stream) {
+  slab_wait_kernel<<<1, 1, 0, stream>>>(flag, target, limit_ns, status);
+  return cudaGetLastError();
+}
 
 // ---------------------------------------------------------------- fixed probe scratch
 // Scratch of the allocation-free probe entry point: a fixed array in the module's global
 // memory, reserved on every device that loads the library until the process exits.  Host
 // code must not pass `g_probe_scratch` itself to a kernel (on the host it names a host-side
-// stand-in); it uses the device address looked up once per device below.
+// stand-in); it passes the device address that cudaGetSymbolAddress returns.
 static __device__ __align__(256) uint4 g_probe_scratch[kStaticProbeScratchBytes / 16];
 
 cudaError_t static_probe_scratch(uint4 **out) {
-  static std::mutex mu;
-  static void *addr[64] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  // Looked up on every call, in the context current on the calling thread: the address
+  // belongs to the module loaded in that context, so a cached value would be wrong for a
+  // caller that switches contexts (cuCtxSetCurrent) or after cudaDeviceReset.  The lookup
+  // allocates nothing; the first one in a context may load the module, so the first call
+  // should precede any stream capture.
+  void *p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_probe_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    // Once per device, with that device current.
-    void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_probe_scratch);
-    if (e != cudaSuccess) return e;
-    addr[dev] = p;
-  }
-  *out = static_cast<uint4 *>(addr[dev]);
+  *out = static_cast<uint4 *>(p);
   return cudaSuccess;
 }
 

@@ -15,6 +15,10 @@ constexpr int kMaxRanks = 16;
 // Default bound of every on-device wait (global-timer nanoseconds).  A healthy wait in any
 // kernel here lasts microseconds; two seconds only ever trips when something is wrong.
 constexpr long long kWaitLimitNs = 2000000000LL;
+// Bound of the waits a CTA runs while shutting down after an abort (for its own copies and
+// MMAs in flight, which end within microseconds).  Kept apart from the caller-set wait limit,
+// so that a short limit never lets a CTA exit before its own asynchronous work has landed.
+constexpr long long kDrainLimitNs = 2000000000LL;
 
 // Bounded wait on an mbarrier phase.  Returns false when the CTA-wide abort flag is set or
 // the limit passes; in the latter case it raises the abort flag and records XS_ERR_TIMEOUT
@@ -72,6 +76,10 @@ struct AttnParams {
   float *lse;              // kPartial: natural-log log-sum-exp of each query row
   unsigned long long *spans;  // kSeqScatterSpans: [n_items][2 tiles][4 warps][3]
   void *dest[kMaxRanks];   // kSeqScatter
+  // kSeqScatter, optional (slab_flags[0] == nullptr: none): per destination slab r, a counter
+  // to which every epilogue warp adds, with a system-scope release after its stores, the
+  // number of rows it stored into dest[r].
+  unsigned int *slab_flags[kMaxRanks];
   int B, H, S, D, P;       // H = heads held by this call (the rank's heads); S = query rows
   int S_kv;                // key/value rows (= S except for partial attention over a shard)
   int H_dest;              // heads per destination row (all heads of the layer)
@@ -83,6 +91,10 @@ struct AttnParams {
   float scale_log2;        // softmax scale * log2(e)
   int *status;
   long long wait_limit_ns;
+  // Self-test only (-1 otherwise): the TMA producer of every CTA stops before its fill number
+  // stall_fill (Q and K/V tile fills counted together), as if a copy never arrived, and the
+  // other roles' bounded waits then run out.
+  int stall_fill;
 };
 
 // Host launchers (attn.cu).
@@ -115,12 +127,18 @@ struct BurstParams {
 };
 cudaError_t launch_burst_probe(const BurstParams &p, int threads, cudaStream_t stream);
 
-// Allocation-free probe: device address of the fixed scratch array on the current device
-// (looked up on the first call per device), and its size.
+// Allocation-free probe: device address of the fixed scratch array in the current context
+// (looked up on every call), and its size.
 constexpr long long kStaticProbeScratchBytes = 32LL << 20;
 cudaError_t static_probe_scratch(uint4 **out);
 
 cudaError_t launch_wait_selftest(int *status, long long limit_ns, cudaStream_t stream);
+
+// Consumer side of the per-slab arrival counters: one thread polls *flag (acquire, system
+// scope) until it has reached target (wrap-around safe), or writes XS_ERR_TIMEOUT to *status
+// after limit_ns.
+cudaError_t launch_slab_wait(const unsigned int *flag, unsigned int target, long long limit_ns,
+                             int *status, cudaStream_t stream);
 
 // ---------------------------------------------------------------- log-sum-exp merge
 constexpr int kMaxParts = 16;

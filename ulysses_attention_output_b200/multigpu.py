@@ -12,7 +12,10 @@ is stored by its owner straight into the slab of the rank that needs it, over NV
 the owner goes on to its next tile (the X-Stage explainer, "FlashAttention-A2A
 (Piggybacking)").  ``complete()`` then orders those stores before anything that reads the
 slabs.  No kernel waits on another GPU: the ordering is a one-element collective enqueued
-after the fused kernel.
+after the fused kernel.  Alternatively ``fused_flags()`` has every storing warp add its row
+count to the owning slab's arrival counter with a system-scope release, and ``wait_slabs()``
+waits (bounded) on this GPU's counters: a consumer of a slab can then start without the
+collective.
 
 The serial form (attention, then a separate exchange) packs the head-major output per
 destination GPU with the library's exchange kernel, moves it with one all-to-all of the
@@ -61,6 +64,18 @@ def slab_table(plan: GpuPlan, bases: list[int], nbytes: int) -> list[int]:
     return [bases[r // plan.slabs_local] + (r % plan.slabs_local) * nbytes for r in range(plan.P)]
 
 
+COUNTER_STRIDE = 256  # bytes between two slabs' arrival counters
+
+
+def counter_table(plan: GpuPlan, bases: list[int], slabs_nbytes: int) -> list[int]:
+    """Address, in this process, of every rank's arrival counter: GPU g keeps the counters of
+    its P/N slabs right after them (``slabs_nbytes`` = P/N slabs), COUNTER_STRIDE apart."""
+    if len(bases) != plan.world:
+        raise ValueError(f"need one base per GPU ({plan.world}), got {len(bases)}")
+    return [bases[r // plan.slabs_local] + slabs_nbytes + (r % plan.slabs_local) * COUNTER_STRIDE
+            for r in range(plan.P)]
+
+
 class XsIpc:
     """CUDA IPC through libxs (``xs_ipc_export`` / ``xs_ipc_open`` / ``xs_ipc_close``)."""
 
@@ -101,9 +116,16 @@ class UlyssesGpu:
         self.ipc = ipc if ipc is not None else XsIpc()
         self.backend = dist.get_backend(group)
         self.slab_nbytes = slab_bytes(B, S, H, D, P)
-        self.slabs = torch.empty((self.plan.slabs_local, B, S // P, H, D), dtype=torch.bfloat16,
-                                 device=self.device)
-        handle, offset = self.ipc.export(self.slabs)
+        # One allocation: this GPU's slabs, then one arrival counter per slab (256 bytes apart),
+        # exported together so that the other GPUs map both.
+        nb_slabs = self.plan.slabs_local * self.slab_nbytes
+        self._buf = torch.empty(nb_slabs + COUNTER_STRIDE * self.plan.slabs_local, dtype=torch.uint8,
+                                device=self.device)
+        self.slabs = self._buf[:nb_slabs].view(torch.bfloat16).view(self.plan.slabs_local, B, S // P, H, D)
+        self.counters = self._buf[nb_slabs:].view(torch.int32)[::COUNTER_STRIDE // 4]
+        self.counters.zero_()
+        self._steps_flagged = 0
+        handle, offset = self.ipc.export(self._buf)
         infos = [None] * self.world
         dist.all_gather_object(infos, (self.rank, handle, offset), group=group)
         self._mapped: list[int] = []
@@ -122,6 +144,7 @@ class UlyssesGpu:
             self._unmap()
             raise
         self.dest = slab_table(self.plan, bases, self.slab_nbytes)
+        self.flag_table = counter_table(self.plan, bases, nb_slabs)
         self._token = torch.zeros(1, dtype=torch.float32, device=self.device)
         self._closed = False
 
@@ -133,6 +156,38 @@ class UlyssesGpu:
         import ulysses_attention_output_b200 as xs
         xs.attn_a2a_fused_rank(q, k, v, self.dest, heads_total=self.H, head_offset=self.plan.head_offset,
                                scale=scale, stream=stream, status=status)
+
+    def fused_flags(self, q, k, v, scale=None, stream=None, status=None):
+        """:meth:`fused` that also adds each slab's stored rows to that slab's arrival counter
+        (on the GPU that owns the slab) with a system-scope release; one step adds
+        ``rows_per_slab`` to every counter once all GPUs' calls have run."""
+        import ulysses_attention_output_b200 as xs
+        xs.attn_a2a_fused_flags(q, k, v, self.dest, self.flag_table, heads_total=self.H,
+                                head_offset=self.plan.head_offset, scale=scale, stream=stream, status=status)
+        self._steps_flagged += 1
+
+    @property
+    def rows_per_slab(self) -> int:
+        """Rows (one head of one sequence position) that one step stores into each slab."""
+        return self.B * (self.S // self.P) * self.H
+
+    def wait_slabs(self, stream=None, status=None, limit_ns: int = 2_000_000_000):
+        """Enqueue on ``stream`` a bounded wait until this GPU's slabs hold every row of every
+        flagged step so far (each counter reaches steps x ``rows_per_slab``): the consumer of
+        a slab may then start on it without a collective.  The waits run on this GPU after its
+        own fused call (stream order) and wait only for the other GPUs' stores; ``status``
+        (int32 CUDA tensor) receives XS_ERR_TIMEOUT if a count is still short after
+        ``limit_ns``.  Overwriting a slab that another GPU still reads is not covered: call
+        ``complete()`` between the last read and the next fused call."""
+        import torch
+
+        import ulysses_attention_output_b200 as xs
+        if status is None:
+            raise ValueError("wait_slabs needs a status tensor")
+        target = self._steps_flagged * self.rows_per_slab
+        for i in range(self.plan.slabs_local):
+            xs.slab_wait(self.counters[i:i + 1], target, limit_ns, status, stream=stream)
+        return target
 
     def complete(self, stream=None):
         """Order every GPU's slab stores enqueued so far before the later work on ``stream``.
