@@ -350,10 +350,12 @@ def fit_capacity(points):
             "one_line_GBps": 1.0 / one[0] if one[0] > 0 else None}
 
 
-def knee_sweep(volumes, k: int = 148, r_guess_gbs: float = 7700.0, ghz_guess: float = 1.9,
-               n_gaps: int = 17, n_bursts: int = 48, drop: int = 8, threads: int = 256,
-               scratch_bytes: int = 2 << 30):
-    """T_iss over G densely through [0, 2 V/R] (R guessed) for each V at K producers."""
+def knee_sweep(volumes, k: int = 148, r_guess_gbs: float = 7700.0, issue_guess_gbs: float = 8600.0,
+               ghz_guess: float = 1.9, n_gaps: int = 17, n_bursts: int = 48, drop: int = 8,
+               threads: int = 256, scratch_bytes: int = 2 << 30):
+    """T_iss over G densely through [0, 2.5 (V/R - V/I)] for each V at K producers: the knee
+    of max(T0_iss, V/R - G) lies at V/R - T0_iss, about V (1/R - 1/I) with I the issue rate
+    (R and I guessed from earlier sweeps; the range only has to contain the knee)."""
     import torch
 
     import ulysses_attention_output_b200 as xs
@@ -361,7 +363,7 @@ def knee_sweep(volumes, k: int = 148, r_guess_gbs: float = 7700.0, ghz_guess: fl
     out = []
     for v in volumes:
         vv = (v // (16 * k)) * 16 * k
-        g_max_cycles = 2.0 * vv / r_guess_gbs * ghz_guess
+        g_max_cycles = 2.5 * vv * (1.0 / r_guess_gbs - 1.0 / issue_guess_gbs) * ghz_guess
         for i in range(n_gaps):
             g = int(round(g_max_cycles * i / (n_gaps - 1)))
             out.append(run_point(xs, torch, scratch, k, vv, g, n_bursts, threads, drop))

@@ -66,14 +66,18 @@ struct Smem {
   static constexpr uint32_t kTile = DCH * kChunkBytes;
   static constexpr uint32_t kQ = 0;                                   // 2 tiles
   static constexpr uint32_t kKV = kQ + 2 * kTile;                     // kStages tiles
-  static constexpr uint32_t kStage = kKV + kStages * kTile;           // 8 warps x 16 rows
+  // P_t: 128 rows x 128 keys bf16 per Q tile, two 128-byte-swizzled panels of 64 keys (the
+  // A operand of P V, K-major); after a work item's last P V it holds the staging rows of the
+  // head-major and partial epilogues of tile t.
+  static constexpr uint32_t kP = kKV + kStages * kTile;
+  static constexpr uint32_t kPTile = 2 * kChunkBytes;
   static constexpr uint32_t kStageRowBytes = DCH * 128;
-  static constexpr uint32_t kStageBytes = 8 * kStageRows * kStageRowBytes;
-  static constexpr uint32_t kRowPtr = kStage + kStageBytes;           // 8 x 16 pointers
+  static_assert(kStageRows * kStageRowBytes <= 4096, "a warp's staging rows must fit in its 32 P rows");
+  static constexpr uint32_t kRowPtr = kP + 2 * kPTile;                // 8 warps x 16 pointers
   static constexpr uint32_t kBars = kRowPtr + 8 * kStageRows * 8;
-  // barriers: q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_done[2] drain
-  //           p_lo[2]
-  static constexpr uint32_t kNumBars = 2 + 2 + kStages + kStages + 2 + 2 + 2 + 1 + 2;
+  // barriers: q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] s_read[2] p_full[2]
+  //           p_free[2] drain
+  static constexpr uint32_t kNumBars = 2 + 2 + kStages + kStages + 2 + 2 + 2 + 2 + 1;
   static constexpr uint32_t kMisc = kBars + kNumBars * 8;             // tmem base, abort flag
   static constexpr uint32_t kTotal = kMisc + 16;
   static constexpr size_t kAlloc = kTotal + 1024;                     // room for alignment
@@ -138,19 +142,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 
   const uint32_t sQ = base_u32 + L::kQ;
   const uint32_t sKV = base_u32 + L::kKV;
+  const uint32_t sP = base_u32 + L::kP;
   const uint32_t bar0 = base_u32 + L::kBars;
   // barrier addresses
   auto q_full = [&](int t) { return bar0 + 8u * (0 + t); };
   auto q_empty = [&](int t) { return bar0 + 8u * (2 + t); };
   auto kv_full = [&](uint32_t s) { return bar0 + 8u * (4 + s); };
   auto kv_empty = [&](uint32_t s) { return bar0 + 8u * (4 + kStages + s); };
+  // S_t = Q_t K_j^T complete (MMA -> softmax)
   auto s_full = [&](int t) { return bar0 + 8u * (4 + 2 * kStages + t); };
-  auto p_full = [&](int t) { return bar0 + 8u * (6 + 2 * kStages + t); };
-  auto o_done = [&](int t) { return bar0 + 8u * (8 + 2 * kStages + t); };
-  const uint32_t drain_bar = bar0 + 8u * (10 + 2 * kStages);
-  // P of keys 0-63 of tile t stored (p_full: all of P): the MMA thread starts P V on that half
-  // while the softmax computes the other.
-  auto p_lo = [&](int t) { return bar0 + 8u * (11 + 2 * kStages + t); };
+  // the softmax of tile t holds S_t in registers: Q K^T of the next key tile may overwrite it
+  auto s_read = [&](int t) { return bar0 + 8u * (6 + 2 * kStages + t); };
+  // P_t written to shared memory (and O_t rescaled if needed): P V may run
+  auto p_full = [&](int t) { return bar0 + 8u * (8 + 2 * kStages + t); };
+  // P V of tile t complete: P_t may be rewritten, O_t read or rescaled (MMA -> softmax)
+  auto p_free = [&](int t) { return bar0 + 8u * (10 + 2 * kStages + t); };
+  const uint32_t drain_bar = bar0 + 8u * (12 + 2 * kStages);
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(base + L::kMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(base + L::kMisc + 4);
 
@@ -162,9 +169,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       ptx::mbar_init(q_full(t), 1);
       ptx::mbar_init(q_empty(t), 1);
       ptx::mbar_init(s_full(t), 1);
-      ptx::mbar_init(p_full(t), 4);  // one arrival per softmax warp
-      ptx::mbar_init(p_lo(t), 4);
-      ptx::mbar_init(o_done(t), 1);
+      ptx::mbar_init(s_read(t), 4);  // one arrival per softmax warp of the tile
+      ptx::mbar_init(p_full(t), 4);
+      ptx::mbar_init(p_free(t), 1);
     }
     for (int s = 0; s < kStages; ++s) {
       ptx::mbar_init(kv_full(s), 1);
@@ -211,18 +218,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           if (t == 0) q_filled0 = static_cast<int>(it);
           else q_filled1 = static_cast<int>(it);
         }
-        for (int j = 0; j < n_kv && ok; ++j) {
-          for (int kv = 0; kv < 2; ++kv) {
-            const uint32_t slot = kv_it % kStages;
-            ok = bounded_wait(kv_empty(slot), ((kv_it / kStages) & 1u) ^ 1u, ctl) && fills++ != p.stall_fill;
-            if (!ok) break;
-            ptx::mbar_arrive_expect_tx(kv_full(slot), L::kTile);
-            const CUtensorMap *tm = kv == 0 ? &p.tm_k : &p.tm_v;
-            for (int c = 0; c < DCH; ++c)
-              ptx::tma_load_3d(sKV + slot * L::kTile + c * kChunkBytes, tm, kv_full(slot), c * 64,
-                               j * 128, bh);
-            ++kv_it;
-          }
+        // K runs one key tile ahead of V: K_0, K_1, V_0, K_2, V_1, ..., K_{n-1}, V_{n-2},
+        // V_{n-1} -- the order in which the MMA thread needs them (Q K_{j+1}^T before P_j V_j).
+        for (int f = 0; f < 2 * n_kv && ok; ++f) {
+          const bool is_k = f == 0 || (f & 1 && (f + 1) / 2 < n_kv);
+          const int j = f == 0 ? 0 : is_k ? (f + 1) / 2 : (f == 2 * n_kv - 1 ? n_kv - 1 : f / 2 - 1);
+          const uint32_t slot = kv_it % kStages;
+          ok = bounded_wait(kv_empty(slot), ((kv_it / kStages) & 1u) ^ 1u, ctl) && fills++ != p.stall_fill;
+          if (!ok) break;
+          ptx::mbar_arrive_expect_tx(kv_full(slot), L::kTile);
+          const CUtensorMap *tm = is_k ? &p.tm_k : &p.tm_v;
+          for (int c = 0; c < DCH; ++c)
+            ptx::tma_load_3d(sKV + slot * L::kTile + c * kChunkBytes, tm, kv_full(slot), c * 64,
+                             j * 128, bh);
+          ++kv_it;
         }
       }
       if (!ok) {
@@ -242,12 +251,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     // warp-uniform) and one elected lane issues each MMA and commit.  Run by lane 0 alone,
     // the same loop left the tensor core idle between MMA groups for long enough to cost
     // up to 15% in a layout with more warps per SM.
+    //
+    // Per key tile j the order is Q_0 K_{j+1}^T, Q_1 K_{j+1}^T (each as soon as that tile's
+    // softmax has read S(j) into registers), then P_0 V_j, P_1 V_j (each as soon as that tile's
+    // P(j) is in shared memory).  S of the next key tile is thus ready before the softmax of
+    // the current one ends, and the softmax never waits for the tensor core's P V + Q K^T of
+    // its own tile in between.
     {
       const int ks_d = (p.D + 15) >> 4;              // K steps of 16 covering the true D
       const uint32_t n_pv = static_cast<uint32_t>(ks_d * 16);   // N of P V (D padded to 16)
       const uint32_t idesc_qk = ptx::idesc_bf16_f32(128, 128, 0);
       const uint32_t idesc_pv = ptx::idesc_bf16_f32(128, n_pv, 1);
-      uint32_t kv_it = 0, it = 0, pc0 = 0, pc1 = 0;
+      uint32_t kv_base = 0, it = 0;
+      uint32_t sr0 = 0, sr1 = 0, pc0 = 0, pc1 = 0;  // s_read / p_full phases consumed per tile
       bool ok = true;
 
       // Descriptors are built once; per MMA only compile-time offsets are added (a per-MMA
@@ -256,7 +272,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       const uint64_t dq0 = ptx::smem_desc_sw128(sQ, 16, 1024);
       const uint64_t dk0 = ptx::smem_desc_sw128(sKV, 16, 1024);
       const uint64_t dv0 = ptx::smem_desc_sw128(sKV, kChunkBytes, 1024);
-      constexpr uint64_t kTileDesc = L::kTile >> 4;  // one tile, in descriptor address units
+      const uint64_t dp0 = ptx::smem_desc_sw128(sP, 16, 1024);
+      constexpr uint64_t kTileDesc = L::kTile >> 4;   // one Q/K/V tile, in descriptor units
+      constexpr uint64_t kPDesc = L::kPTile >> 4;     // one P tile
 
       // Every K step of the padded D (DCH * 64) is issued, also when D is smaller: TMA fills
       // Q and K beyond D with zeros, so those steps add exact zeros to S.  No MMA is issued
@@ -272,90 +290,80 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           ptx::mma_ss_elect(d, a + off, b + off, idesc_qk, ks > 0 ? 1u : 0u);
         }
       };
-      // P V over keys [64 half, 64 half + 64): four K steps of 16 keys.
-      auto issue_pv = [&](int t, uint32_t slot, bool acc, int half) {
+      // O_t (+)= P_t V: A = P_t from shared memory (K-major, 128 keys in two swizzled panels),
+      // B = V tile, MN-major (LBO = distance between 64-column panels, SBO = 8 key rows).
+      auto issue_pv = [&](int t, uint32_t slot, bool acc) {
+        const uint64_t a = dp0 + static_cast<uint64_t>(t) * kPDesc;
         const uint64_t b = dv0 + static_cast<uint64_t>(slot) * kTileDesc;
         const uint32_t d = tmem + col_o(t);
-        const uint32_t a = tmem + col_s(t);
 #pragma unroll
-        for (int ks = 4 * half; ks < 4 * half + 4; ++ks) {
-          // A = P (bf16 pairs in TMEM, 8 columns per 16 keys); B = V tile, MN-major:
-          // LBO = distance between 64-column panels, SBO = 8 key rows.
-          ptx::mma_ts_elect(d, a + ks * 8, b + static_cast<uint64_t>(ks * (2048 >> 4)), idesc_pv,
-                      (acc || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t off = static_cast<uint64_t>(((ks >> 2) * kChunkBytes + (ks & 3) * 32) >> 4);
+          ptx::mma_ss_elect(d, a + off, b + static_cast<uint64_t>(ks * (2048 >> 4)), idesc_pv,
+                            (acc || ks > 0) ? 1u : 0u);
         }
+      };
+      // Ring slot and phase parity of fill number f.  Within an item K_0 is fill 0, K_{j+1}
+      // fill 2j + 1 and V_j fill 2j + 2, except V_{n-1}: fill 2n - 1 (K one key tile ahead).
+      auto slot_of = [](uint32_t f) { return f % kStages; };
+      auto par_of = [](uint32_t f) { return (f / kStages) & 1u; };
+      // Wait (whole warp) for a barrier phase; false when the CTA aborts.
+      auto wait = [&](uint32_t bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, bounded_wait(bar, parity, ctl));
       };
 
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++it) {
-        ok = bounded_wait(q_full(0), it & 1u, ctl) && bounded_wait(q_full(1), it & 1u, ctl);
-        ok = __all_sync(0xffffffffu, ok);
+        ok = wait(q_full(0), it & 1u) && wait(q_full(1), it & 1u);
+        const uint32_t fK0 = kv_base;
+        ok = ok && wait(kv_full(slot_of(fK0)), par_of(fK0));
+        // The previous item's last S_t must have been read before Q_t K_0^T overwrites it.
+        if (ok && it > 0) ok = wait(s_read(0), sr0++ & 1u);
         if (!ok) break;
-        uint32_t slotK = kv_it % kStages;
-        ok = bounded_wait(kv_full(slotK), (kv_it / kStages) & 1u, ctl);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        ++kv_it;
         ptx::tc_fence_after();
-        issue_qk(0, slotK);
+        issue_qk(0, slot_of(fK0));
         ptx::mma_commit_elect(s_full(0));
         if (n_kv == 1) ptx::mma_commit_elect(q_empty(0));
-        issue_qk(1, slotK);
+        if (it > 0) {
+          ok = wait(s_read(1), sr1++ & 1u);
+          if (!ok) break;
+          ptx::tc_fence_after();
+        }
+        issue_qk(1, slot_of(fK0));
         ptx::mma_commit_elect(s_full(1));
-        ptx::mma_commit_elect(kv_empty(slotK));
+        ptx::mma_commit_elect(kv_empty(slot_of(fK0)));
         if (n_kv == 1) ptx::mma_commit_elect(q_empty(1));
 
         for (int j = 0; j < n_kv && ok; ++j) {
-          const uint32_t slotV = kv_it % kStages;
-          ok = bounded_wait(kv_full(slotV), (kv_it / kStages) & 1u, ctl);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          ++kv_it;
-          ok = bounded_wait(p_lo(0), pc0 & 1u, ctl);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          ptx::tc_fence_after();
-          issue_pv(0, slotV, j > 0, 0);
-          ok = bounded_wait(p_full(0), pc0 & 1u, ctl);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          ++pc0;
-          ptx::tc_fence_after();
-          issue_pv(0, slotV, true, 1);
-          const bool more = (j + 1) < n_kv;
-          // The s_full commit after QK_t(j+1) also covers PV_t(j), issued just before it, so
-          // o_done is only needed for the last key tile (the epilogue waits for it).
-          if (!more) ptx::mma_commit_elect(o_done(0));
-          if (more) {
-            slotK = kv_it % kStages;
-            ok = bounded_wait(kv_full(slotK), (kv_it / kStages) & 1u, ctl);
-            ok = __all_sync(0xffffffffu, ok);
+          const uint32_t fV = kv_base + 2 * j + (j + 1 < n_kv ? 2 : 1);
+          if (j + 1 < n_kv) {
+            const uint32_t fK = kv_base + 2 * j + 1;
+            ok = wait(kv_full(slot_of(fK)), par_of(fK)) && wait(s_read(0), sr0++ & 1u);
             if (!ok) break;
-            ++kv_it;
-            // (no tcgen05 fence here: K arrived through TMA, no tensor-memory hand-off)
-            issue_qk(0, slotK);
+            ptx::tc_fence_after();
+            issue_qk(0, slot_of(fK));
             ptx::mma_commit_elect(s_full(0));
             if (j + 2 == n_kv) ptx::mma_commit_elect(q_empty(0));
-          }
-          ok = bounded_wait(p_lo(1), pc1 & 1u, ctl);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          ptx::tc_fence_after();
-          issue_pv(1, slotV, j > 0, 0);
-          ok = bounded_wait(p_full(1), pc1 & 1u, ctl);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          ++pc1;
-          ptx::tc_fence_after();
-          issue_pv(1, slotV, true, 1);
-          if (!more) ptx::mma_commit_elect(o_done(1));
-          ptx::mma_commit_elect(kv_empty(slotV));
-          if (more) {
-            issue_qk(1, slotK);
+            ok = wait(s_read(1), sr1++ & 1u);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            issue_qk(1, slot_of(fK));
             ptx::mma_commit_elect(s_full(1));
-            ptx::mma_commit_elect(kv_empty(slotK));
+            ptx::mma_commit_elect(kv_empty(slot_of(fK)));
             if (j + 2 == n_kv) ptx::mma_commit_elect(q_empty(1));
           }
+          ok = wait(kv_full(slot_of(fV)), par_of(fV)) && wait(p_full(0), pc0++ & 1u);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          issue_pv(0, slot_of(fV), j > 0);
+          ptx::mma_commit_elect(p_free(0));
+          ok = wait(p_full(1), pc1++ & 1u);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          issue_pv(1, slot_of(fV), j > 0);
+          ptx::mma_commit_elect(p_free(1));
+          ptx::mma_commit_elect(kv_empty(slot_of(fV)));
         }
+        kv_base += 2 * static_cast<uint32_t>(n_kv);
       }
       // Every MMA the elected lane issued must be complete before TMEM is released.
       ptx::mma_commit_elect(drain_bar);
@@ -371,10 +379,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const uint32_t tO = tmem + lane_base + col_o(t);
     const float sl2 = p.scale_log2;
     const int D = p.D;
-    uint8_t *stg = base + L::kStage + warp * (kStageRows * L::kStageRowBytes);
+    // This thread's row of P_t (two 64-key panels, 128-byte rows, 16-byte chunks XOR-swizzled
+    // by row % 8, as TMA lays out a Q tile) and, after the item's last P V, the staging rows of
+    // this warp: the 4 KB of panel 0 that hold the warp's own 32 P rows, so that a warp that
+    // has moved on to the next item's P never writes where another still stages.
+    const uint32_t sP_t = sP + static_cast<uint32_t>(t) * L::kPTile;
+    const uint32_t p_row = sP_t + static_cast<uint32_t>(row) * 128u;
+    const uint32_t p_sw = static_cast<uint32_t>(row & 7);
+    uint8_t *stg = base + L::kP + t * L::kPTile + wq * 4096;
     uint8_t **rowptr = reinterpret_cast<uint8_t **>(base + L::kRowPtr) + warp * kStageRows;
-    uint32_t sc = 0;       // s_full phases consumed
-    uint32_t item_cnt = 0;  // work items finished by this CTA (o_done completes once per item)
+    uint32_t sc = 0;    // s_full phases consumed
+    uint32_t npv = 0;   // P V of this tile handed to the MMA thread (p_free completes once each)
     bool ok = true;
 
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
@@ -390,35 +405,32 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         ++sc;
         ptx::tc_fence_after();
         const int kv_valid = p.S_kv - j * 128;  // < 128 only on a ragged last key tile
-        // Pass 1: row maximum over the 128 scores (one TMEM round trip for the whole row; the
-        // scores stay in registers for pass 2).
-        float m0, m1, m2, m3;
+        // Pass 1: the row's 128 scores from TMEM into registers (one round trip); S_t is then
+        // free, and Q K^T of the next key tile may overwrite it while this thread computes.
         uint32_t sr[128];
-        {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) ptx::tmem_ld32(tS + 32 * q, sr + 32 * q);
-          ptx::tmem_wait_ld();
+        for (int q = 0; q < 4; ++q) ptx::tmem_ld32(tS + 32 * q, sr + 32 * q);
+        ptx::tmem_wait_ld();
 #pragma unroll
-          for (int q = 0; q < 4; ++q) ptx::reg_fence32(sr + 32 * q);
-          if (kv_valid < 128) {
+        for (int q = 0; q < 4; ++q) ptx::reg_fence32(sr + 32 * q);
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(s_read(t));  // one arrival per warp
+        if (kv_valid < 128) {
 #pragma unroll
-            for (int c = 0; c < 128; ++c)
-              if (c >= kv_valid) sr[c] = 0xff800000u;  // -inf
-          }
-          m0 = u2f(sr[0]);
-          m1 = u2f(sr[1]);
-          m2 = u2f(sr[2]);
-          m3 = u2f(sr[3]);
-#pragma unroll
-          for (int c = 4; c < 124; c += 8) {
-            m0 = ptx::max3(m0, u2f(sr[c]), u2f(sr[c + 1]));
-            m1 = ptx::max3(m1, u2f(sr[c + 2]), u2f(sr[c + 3]));
-            m2 = ptx::max3(m2, u2f(sr[c + 4]), u2f(sr[c + 5]));
-            m3 = ptx::max3(m3, u2f(sr[c + 6]), u2f(sr[c + 7]));
-          }
-          m0 = ptx::max3(m0, u2f(sr[124]), u2f(sr[125]));
-          m1 = ptx::max3(m1, u2f(sr[126]), u2f(sr[127]));
+          for (int c = 0; c < 128; ++c)
+            if (c >= kv_valid) sr[c] = 0xff800000u;  // -inf
         }
+        float m0 = u2f(sr[0]), m1 = u2f(sr[1]), m2 = u2f(sr[2]), m3 = u2f(sr[3]);
+#pragma unroll
+        for (int c = 4; c < 124; c += 8) {
+          m0 = ptx::max3(m0, u2f(sr[c]), u2f(sr[c + 1]));
+          m1 = ptx::max3(m1, u2f(sr[c + 2]), u2f(sr[c + 3]));
+          m2 = ptx::max3(m2, u2f(sr[c + 4]), u2f(sr[c + 5]));
+          m3 = ptx::max3(m3, u2f(sr[c + 6]), u2f(sr[c + 7]));
+        }
+        m0 = ptx::max3(m0, u2f(sr[124]), u2f(sr[125]));
+        m1 = ptx::max3(m1, u2f(sr[126]), u2f(sr[127]));
         const float mx = ptx::max3(m0, m1, fmaxf(m2, m3)) * sl2;
         bool rescale = false;
         float alpha = 1.f;
@@ -428,53 +440,46 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           m_run = mx;
           rescale = (j > 0);
         }
-        // Pass 2, 32 columns at a time, from the registers of pass 1: p = 2^(s * scale *
-        // log2 e - m) in packed fp32 pairs, rounded to bf16 pairs and stored over the S
-        // columns as P (the P words of chunk c land in columns [16c, 16c+16); the whole row
-        // was read in pass 1).  (Re-reading S from TMEM here, chunk by chunk, was 1.5-2% slower.)
-        // A fixed subset of the pairs uses the FMA-pipe exponential instead of MUFU.
-        // P is handed over in two halves (keys 0-63: p_lo, then all: p_full), so that P V on
-        // the first half runs while the second is computed.
+        // Pass 2 from the registers of pass 1: p = 2^(s * scale * log2 e - m) in packed fp32
+        // pairs, rounded to bf16 pairs (pk[i] = keys 2i, 2i + 1).  A fixed subset of the pairs
+        // uses the FMA-pipe exponential instead of MUFU.
         const uint64_t sl2x2 = ptx::f2x(sl2, sl2);
         const uint64_t negm2 = ptx::f2x(-m_run, -m_run);
         uint64_t lacc0 = 0, lacc1 = 0;  // packed row sums (0 bits == +0.0f)
-        auto exp_chunk = [&](int ch, uint32_t(&sr)[32]) {
-          if (kv_valid < 128) {
+        uint32_t pk[64];
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
-              if (32 * ch + c >= kv_valid) sr[c] = 0xff800000u;
+        for (int c = 0; c < 64; ++c) {
+          const uint64_t x2 = ptx::fma2(ptx::f2x(u2f(sr[2 * c]), u2f(sr[2 * c + 1])), sl2x2, negm2);
+          float p0, p1;
+          if (emulated_pair(c)) {
+            exp2_fma_pair(x2, p0, p1);
+          } else {
+            float x0, x1;
+            ptx::f2x_split(x2, x0, x1);
+            p0 = ptx::ex2(x0);
+            p1 = ptx::ex2(x1);
           }
-          uint32_t pk[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const uint64_t x2 = ptx::fma2(ptx::f2x(u2f(sr[2 * c]), u2f(sr[2 * c + 1])), sl2x2, negm2);
-            float p0, p1;
-            if (emulated_pair(16 * ch + c)) {
-              exp2_fma_pair(x2, p0, p1);
-            } else {
-              float x0, x1;
-              ptx::f2x_split(x2, x0, x1);
-              p0 = ptx::ex2(x0);
-              p1 = ptx::ex2(x1);
-            }
-            pk[c] = ptx::pack_bf16(p0, p1);
-            // Row sum of the bf16-rounded probabilities, i.e. of exactly the weights P V uses.
-            if (c & 1)
-              madd2(lacc1, pk[c]);
-            else
-              madd2(lacc0, pk[c]);
-          }
-          ptx::tmem_st16(tS + 16 * ch, pk);
-        };
-        // The scores of pass 1 are still in registers: no second TMEM load.
-        exp_chunk(0, reinterpret_cast<uint32_t(&)[32]>(sr[0]));
-        exp_chunk(1, reinterpret_cast<uint32_t(&)[32]>(sr[32]));
+          pk[c] = ptx::pack_bf16(p0, p1);
+          // Row sum of the bf16-rounded probabilities, i.e. of exactly the weights P V uses.
+          if (c & 1)
+            madd2(lacc1, pk[c]);
+          else
+            madd2(lacc0, pk[c]);
+        }
+        {
+          float a0, a1, b0, b1;
+          ptx::f2x_split(lacc0, a0, a1);
+          ptx::f2x_split(lacc1, b0, b1);
+          l_run += (a0 + a1) + (b0 + b1);
+        }
+        // P_t and O_t are those of the previous P V of this tile until it completes.
+        if (npv > 0) {
+          ok = bounded_wait(p_free(t), (npv - 1) & 1u, ctl);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          ptx::tc_fence_after();
+        }
         if (__any_sync(0xffffffffu, rescale)) {
-          // O holds P V of the previous key tiles, all complete: PV_t(j-1) was issued before
-          // QK_t(j), whose completion (s_full) this thread has waited for.  Done before any P
-          // of this key tile is handed over (P V of its first half starts at p_lo), after the
-          // first half's exponentials, whose scores no longer need registers.
-          // 16 columns at a time: the second half's scores still occupy 64 registers.
           const float a = rescale ? alpha : 1.f;
 #pragma unroll 1
           for (int cc = 0; cc < DCH * 4; ++cc) {
@@ -486,31 +491,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(u2f(o[i]) * a);
             ptx::tmem_st16(tO + cc * 16, o);
           }
+          ptx::tmem_wait_st();
         }
-        ptx::tmem_wait_st();
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(p_lo(t));  // one arrival per warp
-        exp_chunk(2, reinterpret_cast<uint32_t(&)[32]>(sr[64]));
-        exp_chunk(3, reinterpret_cast<uint32_t(&)[32]>(sr[96]));
-        {
-          float a0, a1, b0, b1;
-          ptx::f2x_split(lacc0, a0, a1);
-          ptx::f2x_split(lacc1, b0, b1);
-          l_run += (a0 + a1) + (b0 + b1);
-        }
-        ptx::tmem_wait_st();
+        // The row of P into shared memory: chunk c (keys 8c .. 8c+7) of panel c / 8 lands at
+        // 16-byte column (c % 8) ^ (row % 8).
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          ptx::st_shared_v4(p_row + static_cast<uint32_t>(c >> 3) * kChunkBytes +
+                                ((static_cast<uint32_t>(c & 7) ^ p_sw) << 4),
+                            pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(p_full(t));  // one arrival per warp
+        ++npv;
       }
       if (!ok) break;
 
       // ---------------------------------------------------------- epilogue
-      ok = bounded_wait(o_done(t), item_cnt & 1u, ctl);  // the item's last P V
+      ok = bounded_wait(p_free(t), (npv - 1) & 1u, ctl);  // the item's last P V
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      ++item_cnt;
       ptx::tc_fence_after();
       // Store-issue span of this warp's share of the tile (kSeqScatterSpans): SM clock before
       // its first store is prepared and after its last store is issued, and the global timer.
