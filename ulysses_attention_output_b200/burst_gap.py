@@ -372,13 +372,14 @@ def knee_sweep(volumes, k: int = 148, r_guess_gbs: float = 7700.0, issue_guess_g
 
 
 def capacity_sweep(volumes, k: int = 148, r_guess_gbs: float = 5000.0, ghz_guess: float = 1.9,
-                   n_bursts: int = 12, drop: int = 4, threads: int = 256,
-                   scratch_bytes: int = 2 << 30):
-    """Single bursts separated by a gap of 3 V/R (R guessed low): every burst starts drained."""
+                   n_bursts: int = 12, drop: int = 4, threads: int = 256):
+    """Single bursts separated by a gap of 3 V/R (R guessed low): every burst starts drained.
+    The scratch ring holds two of the largest bursts (the stores never revisit a line that
+    an earlier burst may still hold in L2)."""
     import torch
 
     import ulysses_attention_output_b200 as xs
-    scratch = torch.empty(scratch_bytes, dtype=torch.uint8, device="cuda")
+    scratch = torch.empty(max(2 << 30, 2 * max(volumes)), dtype=torch.uint8, device="cuda")
     out = []
     for v in volumes:
         vv = (v // (16 * k)) * 16 * k
@@ -431,8 +432,10 @@ def main(argv=None):
         mib = 1 << 20
         kp = knee_sweep([32 * mib, 64 * mib, 96 * mib, 128 * mib], threads=threads)
         held = (96 * mib // (16 * 148)) * 16 * 148
-        cp = capacity_sweep([v * mib for v in (8, 16, 32, 48, 64, 96, 128, 192, 256, 384, 512)],
-                            threads=threads)
+        # A backlog builds at I - R (issue minus drain rate, ~10% of I for local stores), so a
+        # capacity Q near the L2 size shows only in bursts of Q / (1 - R/I), over 1 GiB.
+        cp = capacity_sweep([v * mib for v in (8, 16, 32, 64, 128, 256, 512, 768, 1024, 1536,
+                                               2048, 3072, 4096)], threads=threads, n_bursts=8, drop=2)
         print(json.dumps({"threads_per_producer": threads, "knee_points": kp,
                           "knee": knee_report(kp, held), "capacity_points": cp,
                           "capacity": fit_capacity(cp)}))
