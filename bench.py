@@ -415,21 +415,20 @@ class UlyssesGpus:
         self.relayout()
 
     def e2e(self):
-        """Per step: this GPU's Q, K, V from pinned host memory, the fused call, completion,
-        its slabs back to pinned host memory, and a second completion so that no GPU's next
-        fused call overwrites a slab that is still being copied out."""
+        """Per step through ``LayerHostPipeline``: this GPU's Q, K, V from pinned host memory,
+        copied per head group while the fused calls of the groups before run; completion; its
+        slabs back to pinned host memory; a second completion so that no GPU's next fused call
+        overwrites a slab that is still being copied out."""
         import torch
+
+        from ulysses_attention_output_b200 import multigpu as MG
+        pipe = MG.LayerHostPipeline(self.layer)
         qp, kp, vp = (t.pin_memory() for t in (self.q_h, self.k_h, self.v_h))
         slabs_h = torch.empty(self.layer.slabs.shape, dtype=torch.bfloat16).pin_memory()
-
-        def step():
-            for dev_t, host_t in ((self.q, qp), (self.k, kp), (self.v, vp)):
-                dev_t.copy_(host_t, non_blocking=True)
-            self.fused()
-            slabs_h.copy_(self.layer.slabs, non_blocking=True)
-            self.layer.complete(self.stream)
-        h2d = 3 * self.q.numel() * 2
-        return step, self.status, h2d, slabs_h.numel() * 2, {"overlap": "none (copies, kernel, copies in sequence)"}
+        return (lambda: pipe.run(qp, kp, vp, slabs_h, stream=self.stream), pipe.status, pipe.h2d_bytes,
+                pipe.d2h_bytes, {"head_groups": len(pipe.groups),
+                                 "overlap": "input copies of each head group overlap the other groups' "
+                                            "kernels; slabs copied out after completion"})
 
     def close(self):
         self.layer.close()

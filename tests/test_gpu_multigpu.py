@@ -5,9 +5,11 @@ the host (stream synchronisation + a gloo barrier), so no kernel waits on anothe
 
 Checked bit for bit against the single-process fused call on all heads (itself checked
 against the oracle by the parity tests): the fused multi-process step, the serial step
-(attention, pack, all-to-all, unpack), and the fused step with arrival counters (each
+(attention, pack, all-to-all, unpack), the fused step with arrival counters (each
 process's warps release-add their row counts to the owning process's counters through the
-IPC mapping; the counts must come out exact).  Every slab is filled with NaN bits first, so a
+IPC mapping; the counts must come out exact), and the end-to-end step with pinned host
+buffers (``LayerHostPipeline``: head groups on two compute streams, slabs copied out after
+completion).  Every slab is filled with NaN bits first, so a
 missing store fails the comparison.
 """
 import os
@@ -43,7 +45,7 @@ def _worker(rank, world, port, case, out_q):
     try:
         out_q.put((rank, None, *_steps(case, dev)))
     except Exception as e:  # reported to the parent instead of leaving it waiting
-        out_q.put((rank, repr(e), False, False, -1, 0))
+        out_q.put((rank, repr(e), False, False, False, -1, 0))
         raise
     finally:
         dist.destroy_process_group()
@@ -96,8 +98,25 @@ def _steps(case, dev):
         [int(c) for c in layer.counters.cpu()] == [layer.rows_per_slab] * pl.slabs_local
     st = int(status.item())
     layer.complete()
+
+    # the end-to-end step with host buffers, two head groups on two compute streams, run
+    # twice (the second run reuses every device buffer)
+    pipe = MM.LayerHostPipeline(layer, chunks=2)
+    qh, kh, vh = (t[:, hs].contiguous().pin_memory() for t in (q, k, v))
+    slabs_h = torch.empty(layer.slabs.shape, dtype=torch.bfloat16).pin_memory()
+    pipe_ok = True
+    for _ in range(2):
+        slabs_h.view(torch.int16).fill_(-1)
+        layer.slabs.view(torch.int16).fill_(-1)
+        layer.complete()
+        pipe.run(qh, kh, vh, slabs_h)
+        torch.cuda.synchronize(dev)
+        pipe_ok = pipe_ok and all(torch.equal(slabs_h[i].view(torch.int16), ref[pl.first_slab + i].cpu().view(torch.int16))
+                                  for i in range(pl.slabs_local))
+    st = st or int(pipe.status.item())
+    layer.complete()
     layer.close()
-    return fused_ok, serial_ok and flags_ok, st, len(layer.dest)
+    return fused_ok, serial_ok and flags_ok, pipe_ok, st, len(layer.dest)
 
 
 @pytest.mark.parametrize("case", CASES)
@@ -116,10 +135,11 @@ def test_two_process_fused_exchange_bit_exact(case, cuda_device):
         for p in procs:
             p.join(timeout=120)
     assert [p.exitcode for p in procs] == [0, 0]
-    for rank, err, fused_ok, serial_ok, st, n_dest in res:
+    for rank, err, fused_ok, serial_ok, pipe_ok, st, n_dest in res:
         assert err is None, f"process {rank}: {err}"
         assert st == 0, f"device status {st} on process {rank}"
         assert n_dest == case[4]
         assert fused_ok, f"fused multi-process slabs of process {rank} differ from the single fused call"
         assert serial_ok, (f"serial (or flagged) multi-process slabs or arrival counts of process {rank} "
                            "differ from the single fused call")
+        assert pipe_ok, f"host-buffer pipeline slabs of process {rank} differ from the single fused call"

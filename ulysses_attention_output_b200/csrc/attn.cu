@@ -553,13 +553,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         constexpr int kEB = EPI == kPartial ? 4 : 2;        // bytes per output element
         constexpr int kChunksPerLd = 2 * kEB;                // 16-byte chunks per 32 columns
         const int nch = D * kEB / 16;                        // 16-byte chunks per output row
+        // whole 32-byte pairs of chunks: the row starts on a 32-byte boundary and has an even
+        // number of chunks (bf16 rows only)
+        const bool row32 = kEB == 2 && (nch & 1) == 0 &&
+                           (reinterpret_cast<uintptr_t>(dst_row) & 31u) == 0;
 #pragma unroll
         for (int cc = 0; cc < DCH * 2; ++cc) {
           uint32_t o[32];
           ptx::tmem_ld32(tO + cc * 32, o);
           ptx::tmem_wait_ld();
           ptx::reg_fence32(o);
-          if (dst_row != nullptr) {
+          if (dst_row != nullptr && row32) {
+            // 32-byte stores: every lane writes whole L2 sectors of its row
+#pragma unroll
+            for (int q8 = 0; q8 < kChunksPerLd / 2; ++q8) {
+              const int c = cc * kChunksPerLd + 2 * q8;  // first 16-byte chunk of the pair
+              if (c < nch) {
+                uint32_t w[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                  w[i] = ptx::pack_bf16(u2f(o[16 * q8 + 2 * i]) * inv_l, u2f(o[16 * q8 + 2 * i + 1]) * inv_l);
+                ptx::st_global_v8(dst_row + c * 16, w);
+              }
+            }
+          } else if (dst_row != nullptr) {
 #pragma unroll
             for (int q4 = 0; q4 < kChunksPerLd; ++q4) {
               const int c = cc * kChunksPerLd + q4;  // 16-byte chunk of the output row

@@ -274,3 +274,102 @@ class UlyssesGpu:
         self._unmap()
         dist.barrier(group=self.group)
         self._closed = True
+
+
+class LayerHostPipeline:
+    """End-to-end step of one GPU of the layer with host buffers: this GPU's heads' q, k, v
+    [B, H/N, S, D] from pinned host memory in, this GPU's slabs [P/N, B, S/P, H, D] to pinned
+    host memory out.
+
+    The local heads are split into ``chunks`` groups: the host-to-device copies of a group's
+    q, k, v (input-copy stream) overlap the fused calls of the groups before it (the caller's
+    stream for even groups, a second compute stream for odd ones), each call storing its
+    heads' rows into every GPU's slabs.  After the last group: ``complete()``, the copy of
+    this GPU's slabs to the host, and ``complete()`` again, so that no GPU's next fused call
+    overwrites a slab that is still being copied out.  The slabs cannot be copied out per
+    group as on one GPU: their rows come from every GPU's heads, and only ``complete()``
+    orders the other GPUs' stores.  ``chunks=1`` runs copies, calls and copies in sequence.
+    """
+
+    def __init__(self, layer: UlyssesGpu, chunks: int | None = None, scale=None):
+        import torch
+        self.layer = layer
+        self.scale = scale
+        pl = layer.plan
+        B, S, D = layer.B, layer.S, layer.D
+        hl = pl.heads_local
+        if chunks is None:
+            # about one wave of 256-row work items per group, at most 20 groups (as on one GPU)
+            sms = torch.cuda.get_device_properties(layer.device).multi_processor_count
+            items_per_head = B * ((S + 255) // 256)
+            chunks = max(1, min(20, hl, (hl * items_per_head) // sms))
+        self.chunks = int(chunks)
+        hc = (hl + self.chunks - 1) // self.chunks
+        self.groups = [(h0, min(hl, h0 + hc)) for h0 in range(0, hl, hc)]
+        dev = layer.device
+        self.q = [torch.empty((B, h1 - h0, S, D), dtype=torch.bfloat16, device=dev) for h0, h1 in self.groups]
+        self.k = [torch.empty_like(t) for t in self.q]
+        self.v = [torch.empty_like(t) for t in self.q]
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.s_in = torch.cuda.Stream(device=dev)
+        self.s_k2 = torch.cuda.Stream(device=dev)   # calls of the odd groups
+        self.ev_in = [torch.cuda.Event() for _ in self.groups]     # group's inputs on the device
+        self.ev_kern = [torch.cuda.Event() for _ in self.groups]   # group's call done
+        self._started = False
+
+    @property
+    def in_shape(self):
+        pl = self.layer.plan
+        return (self.layer.B, pl.heads_local, self.layer.S, self.layer.D)
+
+    @property
+    def h2d_bytes(self) -> int:
+        return 3 * sum(t.numel() for t in self.q) * 2
+
+    @property
+    def d2h_bytes(self) -> int:
+        return self.layer.slabs.numel() * 2
+
+    def run(self, q_host, k_host, v_host, slabs_host, stream=None):
+        """Enqueue one step (collective: every GPU of the layer calls it).  ``slabs_host`` is
+        ready once the caller's stream has reached the point where ``run`` returned."""
+        import torch
+
+        import ulysses_attention_output_b200 as xs
+        layer = self.layer
+        s = stream or torch.cuda.current_stream(layer.device)
+        for name, t in (("q_host", q_host), ("k_host", k_host), ("v_host", v_host)):
+            if tuple(t.shape) != self.in_shape or t.dtype != torch.bfloat16 or t.is_cuda \
+                    or not t.is_contiguous() or not t.is_pinned():
+                raise ValueError(f"{name} must be a contiguous pinned CPU bf16 tensor of shape {self.in_shape}")
+        if tuple(slabs_host.shape) != tuple(layer.slabs.shape) or slabs_host.dtype != torch.bfloat16 \
+                or slabs_host.is_cuda or not slabs_host.is_contiguous() or not slabs_host.is_pinned():
+            raise ValueError(f"slabs_host must be a contiguous pinned CPU bf16 tensor of shape "
+                             f"{tuple(layer.slabs.shape)}")
+        start = torch.cuda.Event()
+        start.record(s)
+        self.s_in.wait_event(start)
+        self.s_k2.wait_event(start)
+        pl = layer.plan
+        for g, (h0, h1) in enumerate(self.groups):
+            with torch.cuda.stream(self.s_in):
+                if self._started:
+                    self.s_in.wait_event(self.ev_kern[g])   # the group's buffers are free
+                for b in range(layer.B):   # one contiguous host range per batch entry
+                    self.q[g][b].copy_(q_host[b, h0:h1], non_blocking=True)
+                    self.k[g][b].copy_(k_host[b, h0:h1], non_blocking=True)
+                    self.v[g][b].copy_(v_host[b, h0:h1], non_blocking=True)
+                self.ev_in[g].record(self.s_in)
+            ks = s if g % 2 == 0 else self.s_k2
+            ks.wait_event(self.ev_in[g])
+            xs.attn_a2a_fused_rank(self.q[g], self.k[g], self.v[g], layer.dest, heads_total=layer.H,
+                                   head_offset=pl.head_offset + h0, scale=self.scale, stream=ks,
+                                   status=self.status)
+            self.ev_kern[g].record(ks)
+        self._started = True
+        for g in range(len(self.groups)):
+            s.wait_event(self.ev_kern[g])
+        layer.complete(s)
+        with torch.cuda.stream(s):
+            slabs_host.copy_(layer.slabs, non_blocking=True)
+        layer.complete(s)
