@@ -89,7 +89,7 @@ __device__ __forceinline__ uint32_t f2u(float x) { return __float_as_uint(x); }
 // Column pairs (of 64 per 128-key tile) whose exponentials run on the FMA pipe instead of
 // MUFU: kEmulatedPer16 of every 16 pairs, spread evenly.
 #ifndef XS_EMULATED_PER16
-#define XS_EMULATED_PER16 4  // 3..7 measured: 4 fastest (2-3% ahead of 5, 3 and 6)
+#define XS_EMULATED_PER16 3  // 0..8 measured with the exponential hand-over: 3 fastest (1% ahead of 4)
 #endif
 constexpr int kEmulatedPer16 = XS_EMULATED_PER16;
 __host__ __device__ constexpr bool emulated_pair(int c) {
