@@ -106,14 +106,37 @@ def measured_peaks():
 KERNEL_SOURCES = ("api.cu", "attn.cu", "ptx.cuh", "xs_internal.cuh")
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source without comments and with whitespace collapsed (string literals kept)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == '"' or c == "'":            # string or character literal, copied verbatim
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def source_digest() -> str:
-    """Hash of the attention kernel's sources: a profile summary is only valid for the kernel
-    it measured."""
+    """Hash of the attention kernel's sources, comments and whitespace aside: a profile summary
+    is only valid for the kernel it measured."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "ulysses_attention_output_b200", "csrc")
     for fn in KERNEL_SOURCES:
-        with open(os.path.join(csrc, fn), "rb") as f:
-            h.update(fn.encode() + b"\0" + f.read())
+        with open(os.path.join(csrc, fn), encoding="utf-8") as f:
+            h.update(fn.encode() + b"\0" + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -143,7 +143,7 @@ XS_API xs_status xs_slab_wait(const unsigned int *flag, unsigned int target, lon
  *   spans     : device, 8-byte aligned, [n_items][2][4][3] uint64 with n_items = B * H *
  *               ceil(S / 256) work items of 256 query rows (two 128-row tiles), for each
  *               tile and each of the four warps that store it: SM clock (clock64) before the
- *               warp prepares its first store, SM clock after its last 16-byte store has
+ *               warp prepares its first store, SM clock after its last store has
  *               been issued (not completed), and the global timer (ns) at the first stamp.
  *   spans_len : words available at spans (>= n_items * 24, else XS_ERR_INVALID_ARG).
  * A separate kernel instance: xs_attn_a2a_fused itself records nothing.
