@@ -132,7 +132,7 @@ __device__ __forceinline__ void madd2(uint64_t &acc, uint32_t pk) {
   acc = ptx::f2x(a0, a1);
 }
 
-template <int DCH, int EPI>
+template <int DCH, int EPI, int KSQ>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
   using L = Smem<DCH>;
   extern __shared__ uint8_t smem_raw[];
@@ -281,16 +281,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       constexpr uint64_t kTileDesc = L::kTile >> 4;   // one Q/K/V tile, in descriptor units
       constexpr uint64_t kPDesc = L::kPTile >> 4;     // one P tile
 
-      // Every K step of the padded D (DCH * 64) is issued, also when D is smaller: TMA fills
-      // Q and K beyond D with zeros, so those steps add exact zeros to S.  No MMA is issued
-      // under a run-time condition (instances of this kernel that did so computed a wrong S
-      // for D = 72 .. 112 in some builds).
+      // KSQ K steps of 16 are issued: every K step of the padded D (DCH * 64), except in the
+      // instance for D <= 80, which issues 5.  TMA fills Q and K beyond D with zeros, so the
+      // steps past D add exact zeros to S.  The count is a compile-time constant; no MMA is
+      // issued under a run-time condition (instances of this kernel that did so computed a
+      // wrong S for D = 72 .. 112 in some builds).
       auto issue_qk = [&](int t, uint32_t slot) {
         const uint64_t a = dq0 + static_cast<uint64_t>(t) * kTileDesc;
         const uint64_t b = dk0 + static_cast<uint64_t>(slot) * kTileDesc;
         const uint32_t d = tmem + col_s(t);
 #pragma unroll
-        for (int ks = 0; ks < DCH * 4; ++ks) {
+        for (int ks = 0; ks < KSQ; ++ks) {
           const uint64_t off = static_cast<uint64_t>(((ks >> 2) * kChunkBytes + (ks & 3) * 32) >> 4);
           ptx::mma_ss_elect(d, a + off, b + off, idesc_qk, ks > 0 ? 1u : 0u);
         }
@@ -717,7 +718,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   }
 }
 
-template <int DCH, int EPI>
+template <int DCH, int EPI, int KSQ = DCH * 4>
 cudaError_t launch_impl(const AttnParams &p, cudaStream_t stream) {
   using L = Smem<DCH>;
   static_assert(L::kAlloc <= 232448, "shared memory budget exceeded");
@@ -731,14 +732,14 @@ cudaError_t launch_impl(const AttnParams &p, cudaStream_t stream) {
   static std::once_flag once[kMaxDevices];
   static cudaError_t setup[kMaxDevices];
   std::call_once(once[dev], [dev] {
-    setup[dev] = cudaFuncSetAttribute(attn_fwd_kernel<DCH, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    setup[dev] = cudaFuncSetAttribute(attn_fwd_kernel<DCH, EPI, KSQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       static_cast<int>(L::kAlloc));
   });
   if (setup[dev] != cudaSuccess) return setup[dev];
   const int sms = device_sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
   const int grid = p.n_items < sms ? p.n_items : sms;
-  attn_fwd_kernel<DCH, EPI><<<grid, kThreads, L::kAlloc, stream>>>(p);
+  attn_fwd_kernel<DCH, EPI, KSQ><<<grid, kThreads, L::kAlloc, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -754,6 +755,10 @@ cudaError_t launch_attention(const AttnParams &p, int epilogue, cudaStream_t str
     return epilogue == kHeadMajor  ? launch_impl<1, kHeadMajor>(p, stream)
            : epilogue == kPartial ? launch_impl<1, kPartial>(p, stream)
                                   : launch_impl<1, kSeqScatter>(p, stream);
+  if (p.D <= 80)  // 5 K steps of Q K^T carry the head dimension (the last one partly zero fill)
+    return epilogue == kHeadMajor  ? launch_impl<2, kHeadMajor, 5>(p, stream)
+           : epilogue == kPartial ? launch_impl<2, kPartial, 5>(p, stream)
+                                  : launch_impl<2, kSeqScatter, 5>(p, stream);
   return epilogue == kHeadMajor  ? launch_impl<2, kHeadMajor>(p, stream)
          : epilogue == kPartial ? launch_impl<2, kPartial>(p, stream)
                                 : launch_impl<2, kSeqScatter>(p, stream);
